@@ -1,0 +1,188 @@
+"""CPU oracle for the DSA layer stack under IndexCache (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps ``dsa_oracle.c`` (plain C,
+IEEE double, single-threaded) through ctypes and shares nothing with the CUDA
+library.  bf16 tensors are passed as their uint16 bit patterns.
+
+Sources: "读懂 IndexCache：从 DSA 的选词开销到跨层索引复用" (IndexCache
+explainer, cited as [IC]) and "注意力机制中的 Index：从位置下标到预算检索"
+(cited as [IDX]); each wrapper names the section it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile dsa_oracle.c into liboracle.so next to it (gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+            "-Wall", "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_indexer_row.argtypes = [P, P, P, i32, i32, i32, P]
+        lib.oracle_indexer_row.restype = ctypes.c_longlong
+        lib.oracle_topk_row.argtypes = [P, i32, i32, P]
+        lib.oracle_topk_row.restype = i32
+        lib.oracle_sparse_attn_row.argtypes = [P, P, i64, P, i64, P, i32, i32, i32, i32, f64, P, P]
+        lib.oracle_sparse_attn_row.restype = i32
+        lib.oracle_dense_attn_row.argtypes = [P, P, i64, P, i64, i32, i32, i32, i32, f64, P, P]
+        lib.oracle_dense_attn_row.restype = None
+        lib.oracle_masked_attn_row.argtypes = [P, P, i64, P, i64, P, i32, i32, i32, i32, i32, i32, f64, P, P]
+        lib.oracle_masked_attn_row.restype = None
+        lib.oracle_indexcache_forward.argtypes = [
+            ctypes.c_char_p, i32, P, P, P, P, P, i64, P, i64, i32, i32, i32, i32,
+            i32, i32, i32, i32, i32, i32, f64, P, P, P, P]
+        lib.oracle_indexcache_forward.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 tensors are passed as uint16 bit patterns")
+    return a
+
+
+def indexer_row(q_row, k, w_row, T: int) -> np.ndarray:
+    """[IDX] §4 index score: I[s] = sum_j w[j] * ReLU(q[j] . k[s]) for s < T.
+
+    q_row [H, d] bf16 bits, k [>=T, d] bf16 bits, w_row [H] float32."""
+    q_row, k = _bits(q_row), _bits(k)
+    w_row = np.ascontiguousarray(w_row, dtype=np.float32)
+    H, d = q_row.shape
+    assert k.shape[1] == d and k.shape[0] >= T and w_row.shape == (H,)
+    out = np.zeros(max(T, 1), dtype=np.float64)
+    _load().oracle_indexer_row(_p(q_row), _p(k), _p(w_row), H, d, T, _p(out))
+    return out[:T]
+
+
+def topk_row(I, T: int, k: int) -> np.ndarray:
+    """[IDX] §4 TopK over s < T; ties -> lower s; ascending s then -1 pad."""
+    I = np.ascontiguousarray(I, dtype=np.float64)
+    assert I.shape[0] >= T
+    out = np.empty(k, dtype=np.int32)
+    _load().oracle_topk_row(_p(I), T, k, _p(out))
+    return out
+
+
+def _attn_args(q_row, K, V):
+    q_row, K, V = _bits(q_row), _bits(K), _bits(V)
+    assert K.ndim == 2 and V.ndim == 2
+    return q_row, K, V
+
+
+def sparse_attn_row(q_row, K, V, idx, scale: float, Dv: int | None = None):
+    """[IDX] §2 alpha-hat / o-hat over the selected set.  Returns (out, lse).
+
+    q_row [n_h, Dqk]; K [Lk, >=Dqk] and V [Lk, >=Dv] (row-major; V may be a
+    column view of the same latent rows); idx [k] int32 with -1 padding."""
+    q_row, K, V = _attn_args(q_row, K, V)
+    n_h, Dqk = q_row.shape
+    Dv = V.shape[1] if Dv is None else Dv
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    out = np.zeros((n_h, Dv), dtype=np.float64)
+    lse = np.zeros(n_h, dtype=np.float64)
+    _load().oracle_sparse_attn_row(_p(q_row), _p(K), K.shape[1], _p(V), V.shape[1],
+                                   _p(idx), idx.shape[0], n_h, Dqk, Dv, scale,
+                                   _p(out), _p(lse))
+    return out, lse
+
+
+def dense_attn_row(q_row, K, V, T: int, scale: float, Dv: int | None = None):
+    """[IDX] §1 dense causal attention over P_t = {s < T}.  Returns (out, lse)."""
+    q_row, K, V = _attn_args(q_row, K, V)
+    n_h, Dqk = q_row.shape
+    Dv = V.shape[1] if Dv is None else Dv
+    out = np.zeros((n_h, Dv), dtype=np.float64)
+    lse = np.zeros(n_h, dtype=np.float64)
+    _load().oracle_dense_attn_row(_p(q_row), _p(K), K.shape[1], _p(V), V.shape[1], T,
+                                  n_h, Dqk, Dv, scale, _p(out), _p(lse))
+    return out, lse
+
+
+def masked_attn_row(q_row, K, V, idx, T: int, scale: float, Dv: int | None = None):
+    """[IDX] §6.4 index-mask formulation (-inf scatter + causal mask)."""
+    q_row, K, V = _attn_args(q_row, K, V)
+    n_h, Dqk = q_row.shape
+    Dv = V.shape[1] if Dv is None else Dv
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    out = np.zeros((n_h, Dv), dtype=np.float64)
+    lse = np.zeros(n_h, dtype=np.float64)
+    _load().oracle_masked_attn_row(_p(q_row), _p(K), K.shape[1], _p(V), V.shape[1],
+                                   _p(idx), idx.shape[0], T, K.shape[0], n_h, Dqk, Dv,
+                                   scale, _p(out), _p(lse))
+    return out, lse
+
+
+def _ptr_array(arrs):
+    arr = (ctypes.c_void_p * len(arrs))()
+    for i, a in enumerate(arrs):
+        arr[i] = None if a is None else a.ctypes.data
+    return arr
+
+
+def indexcache_forward(pattern: str, layers, *, B, Lq, Lk, start_pos, H, dI, k,
+                       n_h, Dqk, Dv, scale, kv_cols_k=None, kv_cols_v=None):
+    """[IC] §1.1-§1.2 (Figure 2 loop) over whole small inputs.
+
+    ``layers`` is a list of dicts with keys q_idx, k_idx, w (F layers; may be
+    None on S layers), q, and either kv (MLA latent rows: K = all columns, V
+    = the first Dv columns) or k and v.  Returns (idx [L,B,Lq,k] int32,
+    out [L,B,Lq,n_h,Dv] f64, lse [L,B,Lq,n_h] f64, counters dict) or raises
+    ValueError for an invalid pattern."""
+    n = len(layers)
+    keep = []
+    qi, ki, wi, qq, KK, VV = [], [], [], [], [], []
+    ks = vs = None
+    for L in layers:
+        if L.get("q_idx") is not None:
+            a, b_, c = _bits(L["q_idx"]), _bits(L["k_idx"]), np.ascontiguousarray(L["w"], np.float32)
+            keep += [a, b_, c]
+            qi.append(a); ki.append(b_); wi.append(c)
+        else:
+            qi.append(None); ki.append(None); wi.append(None)
+        q = _bits(L["q"]); keep.append(q); qq.append(q)
+        if "kv" in L:
+            kv = _bits(L["kv"]); keep.append(kv)
+            KK.append(kv); VV.append(kv)
+            ks = vs = kv.shape[-1]
+        else:
+            K_, V_ = _bits(L["k"]), _bits(L["v"]); keep += [K_, V_]
+            KK.append(K_); VV.append(V_)
+            ks, vs = K_.shape[-1], V_.shape[-1]
+    idx = np.zeros((n, B, Lq, k), dtype=np.int32)
+    out = np.zeros((n, B, Lq, n_h, Dv), dtype=np.float64)
+    lse = np.zeros((n, B, Lq, n_h), dtype=np.float64)
+    counters = np.zeros(2, dtype=np.int64)
+    rc = _load().oracle_indexcache_forward(
+        pattern.encode(), n, _ptr_array(qi), _ptr_array(ki), _ptr_array(wi),
+        _ptr_array(qq), _ptr_array(KK), ks, _ptr_array(VV), vs, B, Lq, Lk,
+        start_pos, H, dI, k, n_h, Dqk, Dv, scale, _ptr_array(list(idx)),
+        _ptr_array(list(out)), _ptr_array(list(lse)), _p(counters))
+    if rc != 0:
+        raise ValueError(f"invalid IndexCache pattern {pattern!r}")
+    return idx, out, lse, {"indexer_calls": int(counters[0]), "scored_pairs": int(counters[1])}

@@ -1,0 +1,361 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other
+than itself -- a hand-worked example, a closed form, a special case that
+reduces to a textbook/library routine, an invariant, or brute force on tiny
+inputs.  CPU only."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_13_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(x):
+    return synth.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def f32(b):
+    return synth.bf16_bits_to_f32(b).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# indexer: I[t,s] = sum_j w_j ReLU(q_j . k_s)
+
+
+def test_indexer_hand_example(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "indexer_hand_example.json")))
+    q, k = bf16(g["q"]), bf16(g["k"])
+    I = oracle_mod.indexer_row(q, k, np.array(g["w"], np.float32), g["T"])
+    assert I.tolist() == g["scores"]
+    for kk, want in g["topk"].items():
+        assert oracle_mod.topk_row(I, g["T"], int(kk)).tolist() == want
+
+
+def test_indexer_single_head_is_relu_dot(oracle_mod):
+    # H = 1, w = 1 reduces to ReLU of a plain matrix-vector product.
+    rng = np.random.default_rng(0)
+    q = bf16(rng.normal(size=(1, 32)))
+    k = bf16(rng.normal(size=(40, 32)))
+    I = oracle_mod.indexer_row(q, k, np.ones(1, np.float32), 37)
+    ref = np.maximum(f32(k)[:37] @ f32(q)[0], 0.0)
+    np.testing.assert_allclose(I, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_indexer_linear_regime_folds_heads(oracle_mod):
+    # All q, k >= 0: every dot is >= 0, ReLU is the identity and the head sum
+    # folds into one combined query sum_j w_j q_j (catches transposed or
+    # mis-indexed heads, a dropped weight, or a wrong key row).
+    rng = np.random.default_rng(1)
+    H, d, T = 6, 16, 25
+    q = bf16(np.abs(rng.normal(size=(H, d))))
+    k = bf16(np.abs(rng.normal(size=(T + 3, d))))
+    w = rng.normal(size=H).astype(np.float32)
+    I = oracle_mod.indexer_row(q, k, w, T)
+    qc = (w.astype(np.float64)[:, None] * f32(q)).sum(0)
+    np.testing.assert_allclose(I, f32(k)[:T] @ qc, rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_negative_dots_give_zero(oracle_mod):
+    # q >= 0, k <= 0: every dot <= 0, so ReLU zeroes all heads (a sign error
+    # in the ReLU would make the scores non-zero).
+    rng = np.random.default_rng(2)
+    q = bf16(np.abs(rng.normal(size=(4, 8))) + 0.1)
+    k = bf16(-np.abs(rng.normal(size=(10, 8))) - 0.1)
+    I = oracle_mod.indexer_row(q, k, rng.normal(size=4).astype(np.float32), 10)
+    assert np.all(I == 0.0)
+
+
+def test_indexer_integer_inputs_exact(oracle_mod):
+    # Integer q/k in [-4,4] and w = +-2^-m: every score is a multiple of 1/8
+    # and |I| <= 64 * 2048, so the double result must be exactly the integer
+    # arithmetic result computed here with Python ints.
+    rng = np.random.default_rng(3)
+    H, d, T = 5, 12, 9
+    qi = rng.integers(-4, 5, size=(H, d))
+    ki = rng.integers(-4, 5, size=(T, d))
+    m = rng.integers(0, 4, size=H)
+    sgn = rng.choice([-1, 1], size=H)
+    w = (sgn * 2.0 ** (-m)).astype(np.float32)
+    I = oracle_mod.indexer_row(bf16(qi), bf16(ki), w, T)
+    for s in range(T):
+        acc8 = 0  # score * 8 as an exact integer
+        for j in range(H):
+            dot = int(sum(int(qi[j, c]) * int(ki[s, c]) for c in range(d)))
+            acc8 += int(sgn[j]) * (8 >> int(m[j])) * max(dot, 0)
+        assert I[s] * 8 == acc8
+
+
+def test_indexer_positive_homogeneity_in_w(oracle_mod):
+    rng = np.random.default_rng(4)
+    q, k = bf16(rng.normal(size=(3, 8))), bf16(rng.normal(size=(12, 8)))
+    w = rng.normal(size=3).astype(np.float32)
+    I1 = oracle_mod.indexer_row(q, k, w, 12)
+    I4 = oracle_mod.indexer_row(q, k, (4 * w).astype(np.float32), 12)
+    np.testing.assert_array_equal(I4, 4 * I1)
+
+
+# --------------------------------------------------------------------------
+# top-k
+
+
+def _rank_select(I, T, k):
+    """Brute force: s is selected iff fewer than k candidates beat it, where
+    u beats s when I[u] > I[s] or (I[u] == I[s] and u < s)."""
+    sel = []
+    for s in range(T):
+        beats = sum(1 for u in range(T) if I[u] > I[s] or (I[u] == I[s] and u < s))
+        if beats < k:
+            sel.append(s)
+    return sel + [-1] * (k - len(sel))
+
+
+@pytest.mark.parametrize("T,k", [(0, 4), (1, 4), (3, 4), (4, 4), (9, 4), (40, 7), (64, 64), (65, 64)])
+def test_topk_matches_rank_brute_force(oracle_mod, T, k):
+    rng = np.random.default_rng(T * 131 + k)
+    I = rng.integers(-3, 4, size=max(T, 1)).astype(np.float64)  # many ties
+    got = oracle_mod.topk_row(I, T, k).tolist()
+    assert got == _rank_select(I, T, k)
+
+
+def test_topk_all_equal_takes_lowest_positions(oracle_mod):
+    I = np.zeros(100)
+    assert oracle_mod.topk_row(I, 100, 8).tolist() == list(range(8))
+
+
+def test_topk_negative_zero_ties_positive_zero(oracle_mod):
+    I = np.array([-0.0, 0.0, -0.0, 0.0, -1.0])
+    assert oracle_mod.topk_row(I, 5, 2).tolist() == [0, 1]
+
+
+def test_topk_negative_weights_pick_smallest_relu(oracle_mod):
+    # With every head weight negative, I = -sum |w_j| ReLU(.), so the top-k
+    # are the positions with the smallest non-negative ReLU mass.
+    rng = np.random.default_rng(5)
+    q = bf16(rng.normal(size=(1, 16)))
+    k = bf16(rng.normal(size=(50, 16)))
+    I = oracle_mod.indexer_row(q, k, np.array([-1.0], np.float32), 50)
+    relu = np.maximum(f32(k) @ f32(q)[0], 0.0)
+    order = sorted(range(50), key=lambda s: (relu[s], s))[:10]
+    assert oracle_mod.topk_row(I, 50, 10).tolist() == sorted(order)
+
+
+# --------------------------------------------------------------------------
+# sparse / dense / masked attention
+
+
+def _attn_inputs(seed, T, n_h=4, D=16, Dv=8):
+    rng = np.random.default_rng(seed)
+    q = bf16(rng.normal(size=(n_h, D)))
+    K = bf16(rng.normal(size=(T, D)))
+    V = bf16(rng.normal(size=(T, Dv)))
+    return q, K, V
+
+
+def test_attention_golden_closed_form(oracle_mod):
+    # q = (1, 0), keys give logits 0, 1, 2; V = (1,0), (0,1), (1,1).
+    q = bf16([[1, 0]])
+    K = bf16([[0, 7], [1, -3], [2, 5]])
+    V = bf16([[1, 0], [0, 1], [1, 1]])
+    e = math.e
+    out, lse = oracle_mod.dense_attn_row(q, K, V, 3, 1.0)
+    z = 1 + e + e * e
+    np.testing.assert_allclose(out[0], [(1 + e * e) / z, (e + e * e) / z], rtol=1e-14)
+    np.testing.assert_allclose(lse[0], math.log(z), rtol=1e-14)
+    out, lse = oracle_mod.sparse_attn_row(q, K, V, np.array([0, 2, -1], np.int32), 1.0)
+    np.testing.assert_allclose(out[0], [1.0, e * e / (1 + e * e)], rtol=1e-14)
+    np.testing.assert_allclose(lse[0], math.log(1 + e * e), rtol=1e-14)
+
+
+def test_dense_attention_matches_torch_sdpa(oracle_mod):
+    T, n_h, D, Dv = 23, 3, 16, 8
+    q, K, V = _attn_inputs(6, T + 1, n_h, D, Dv)
+    scale = 0.3
+    out, _ = oracle_mod.dense_attn_row(q, K, V, T, scale)
+    qt = torch.tensor(f32(q))[None, :, None, :]            # [1, H, 1, D]
+    kt = torch.tensor(f32(K)[:T])[None, None].expand(1, n_h, T, D)
+    vt = torch.tensor(f32(V)[:T])[None, None].expand(1, n_h, T, Dv)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+    np.testing.assert_allclose(out, ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("T,k", [(1, 4), (5, 8), (8, 8), (30, 64)])
+def test_sparse_equals_dense_when_k_covers_history(oracle_mod, T, k):
+    q, K, V = _attn_inputs(T, T + 2)
+    I = np.random.default_rng(T).normal(size=T)
+    idx = oracle_mod.topk_row(I, T, k)
+    a, la = oracle_mod.sparse_attn_row(q, K, V, idx, 0.25)
+    b, lb = oracle_mod.dense_attn_row(q, K, V, T, 0.25)
+    np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(la, lb, rtol=1e-13)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_mask_formulation_equals_sparse(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    T, Lk, k = 40, 48, 12
+    q, K, V = _attn_inputs(seed + 10, Lk)
+    idx = np.sort(rng.choice(T, size=9, replace=False)).astype(np.int32)
+    idx = np.concatenate([idx, -np.ones(k - 9, np.int32)])
+    a, la = oracle_mod.sparse_attn_row(q, K, V, idx, 0.5)
+    b, lb = oracle_mod.masked_attn_row(q, K, V, idx, T, 0.5)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(la, lb, rtol=1e-12)
+
+
+def test_sparse_error_bound_holds_at_every_t(oracle_mod):
+    # ||o_t - o_hat_t|| <= 2 V R_t(S_t), with V = max ||v_s|| and R_t the dense
+    # attention mass outside S_t.
+    T_max, n_h, D, Dv, k = 48, 2, 8, 8, 6
+    q_all = [_attn_inputs(100 + t, 1, n_h, D, Dv)[0] for t in range(T_max)]
+    _, K, V = _attn_inputs(7, T_max, n_h, D, Dv)
+    Vf = f32(V)
+    rng = np.random.default_rng(8)
+    scale = 0.7
+    for t in range(1, T_max):
+        I = rng.normal(size=t)
+        idx = oracle_mod.topk_row(I, t, k)
+        o_hat, _ = oracle_mod.sparse_attn_row(q_all[t], K, V, idx, scale)
+        o, _ = oracle_mod.dense_attn_row(q_all[t], K, V, t, scale)
+        Vmax = np.linalg.norm(Vf[:t], axis=1).max()
+        sel = set(int(s) for s in idx if s >= 0)
+        for h in range(n_h):
+            e = scale * (f32(K)[:t] @ f32(q_all[t])[h])
+            a = np.exp(e - e.max()); a /= a.sum()
+            R = sum(a[s] for s in range(t) if s not in sel)
+            assert np.linalg.norm(o[h] - o_hat[h]) <= 2 * Vmax * R + 1e-12
+
+
+def test_single_row_and_uniform_logits(oracle_mod):
+    q, K, V = _attn_inputs(9, 20)
+    out, lse = oracle_mod.sparse_attn_row(q, K, V, np.array([-1, 7, -1], np.int32), 1.0)
+    np.testing.assert_array_equal(out, np.tile(f32(V)[7], (q.shape[0], 1)))
+    np.testing.assert_allclose(lse, 1.0 * (f32(q) @ f32(K)[7]), rtol=1e-14)
+    zero_q = bf16(np.zeros((2, 16)))
+    sel = np.array([3, 11, 19, 2], np.int32)
+    out, lse = oracle_mod.sparse_attn_row(zero_q, K, V, sel, 1.0)
+    np.testing.assert_allclose(out[0], f32(V)[sel].mean(0), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lse, math.log(4), rtol=1e-14)
+
+
+def test_empty_selection_gives_zero(oracle_mod):
+    q, K, V = _attn_inputs(10, 4)
+    out, lse = oracle_mod.sparse_attn_row(q, K, V, -np.ones(5, np.int32), 1.0)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_selection_order_does_not_matter(oracle_mod):
+    q, K, V = _attn_inputs(11, 30)
+    idx = np.array([4, 9, 17, 22, -1, -1], np.int32)
+    a, _ = oracle_mod.sparse_attn_row(q, K, V, idx, 0.5)
+    b, _ = oracle_mod.sparse_attn_row(q, K, V, np.array([-1, 22, 4, -1, 17, 9], np.int32), 0.5)
+    np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# the IndexCache layer loop
+
+
+def _stack(seed, pattern, B=2, L=24, H=3, dI=8, n_h=2, D=8, Dv=4, int_idx=True):
+    layers = []
+    for l in range(len(pattern)):
+        # indexer inputs exist on every layer; the loop reads them on F layers only
+        ent = {}
+        ent["q_idx"] = synth.tensor(seed, synth.Q_IDX, synth.INT9, l, (B, L, H, dI))
+        ent["k_idx"] = synth.tensor(seed, synth.K_IDX, synth.INT9, l, (B, L, dI))
+        ent["w"] = synth.tensor(seed, synth.W, synth.POW2W, l, (B, L, H), bf16=False)
+        ent["q"] = synth.tensor(seed, synth.Q, synth.NORMAL, l, (B, L, n_h, D), sigma=0.5)
+        ent["k"] = synth.tensor(seed, synth.K_SEP, synth.NORMAL, l, (B, L, D), sigma=0.5)
+        ent["v"] = synth.tensor(seed, synth.V_SEP, synth.NORMAL, l, (B, L, Dv), sigma=0.5)
+        layers.append(ent)
+    dims = dict(B=B, Lq=L, Lk=L, start_pos=0, H=H, dI=dI, k=5, n_h=n_h, Dqk=D, Dv=Dv,
+                scale=1 / math.sqrt(D))
+    return layers, dims
+
+
+def test_pattern_validation_and_reuse_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "fsssfsss_reuse.json")))
+    layers, dims = _stack(0, g["pattern"])
+    idx, out, lse, cnt = oracle_mod.indexcache_forward(g["pattern"], layers, **dims)
+    assert cnt["indexer_calls"] == g["indexer_runs"]
+    for l, src in enumerate(g["source_layer_zero_based"]):
+        np.testing.assert_array_equal(idx[l], idx[src])
+    # layers 0 and 4 run their own indexers on different inputs
+    assert not np.array_equal(idx[0], idx[4])
+    for bad in g["invalid_patterns"]:
+        n = max(len(bad), 1)
+        with pytest.raises(ValueError):
+            oracle_mod.indexcache_forward(bad, (layers * 2)[:n] if bad else layers[:1], **dims)
+
+
+def test_all_f_equals_per_layer_dsa(oracle_mod):
+    pattern = "FFF"
+    layers, d = _stack(1, pattern)
+    idx, out, lse, _ = oracle_mod.indexcache_forward(pattern, layers, **d)
+    for l, L in enumerate(layers):
+        for b in range(d["B"]):
+            for i in range(d["Lq"]):
+                I = oracle_mod.indexer_row(L["q_idx"][b, i], L["k_idx"][b], L["w"][b, i], i)
+                sel = oracle_mod.topk_row(I, i, d["k"])
+                np.testing.assert_array_equal(idx[l, b, i], sel)
+                o, _ = oracle_mod.sparse_attn_row(L["q"][b, i], L["k"][b], L["v"][b], sel, d["scale"])
+                np.testing.assert_array_equal(out[l, b, i], o)
+
+
+def test_shared_layer_uses_own_kv_at_cached_positions(oracle_mod):
+    # [IC] §1.2: an S layer reads the F layer's positions but its OWN K/V.
+    layers, d = _stack(2, "FS")
+    idx, out, _, _ = oracle_mod.indexcache_forward("FS", layers, **d)
+    np.testing.assert_array_equal(idx[0], idx[1])
+    assert not np.allclose(out[0], out[1])
+    b, i = 1, 17
+    o, _ = oracle_mod.sparse_attn_row(layers[1]["q"][b, i], layers[1]["k"][b], layers[1]["v"][b],
+                                      idx[0, b, i], d["scale"])
+    np.testing.assert_array_equal(out[1, b, i], o)
+
+
+def test_first_row_attends_nothing(oracle_mod):
+    layers, d = _stack(3, "F")
+    idx, out, lse, _ = oracle_mod.indexcache_forward("F", layers, **d)
+    assert np.all(idx[0, :, 0] == -1)
+    assert np.all(out[0, :, 0] == 0) and np.all(np.isneginf(lse[0, :, 0]))
+    # row i sees exactly min(i, k) positions, all < i
+    for i in range(d["Lq"]):
+        sel = idx[0, 0, i]
+        valid = sel[sel >= 0]
+        assert len(valid) == min(i, d["k"]) and np.all(valid < i)
+        assert np.all(np.diff(valid) > 0)
+
+
+@pytest.mark.parametrize("N", [4, 8, 16])
+def test_indexer_work_scales_as_m_over_n(oracle_mod, N):
+    # [IC] §1.2: keeping M of N indexers takes prefill indexer work from
+    # O(N L^2) to O(M L^2); the oracle counts every scored (t, s) pair.
+    L = 10
+    pairs_per_layer = L * (L - 1) // 2
+    for pat, M in [("F" * N, N), ("FS" * (N // 2), N // 2), ("FSSS" * (N // 4), N // 4)]:
+        layers, d = _stack(4, pat, B=1, L=L, H=2, dI=4, n_h=1, D=4, Dv=4)
+        _, _, _, cnt = oracle_mod.indexcache_forward(pat, layers, **d)
+        assert cnt["indexer_calls"] == M
+        assert cnt["scored_pairs"] == M * pairs_per_layer
+
+
+def test_decode_rows_use_start_pos(oracle_mod):
+    # Lq = 1 query at absolute position start_pos = Lk sees every cached key.
+    B, Lk, H, dI = 1, 30, 2, 8
+    qi = synth.tensor(5, synth.Q_IDX, synth.INT9, 0, (B, 1, H, dI))
+    ki = synth.tensor(5, synth.K_IDX, synth.INT9, 0, (B, Lk, dI))
+    w = synth.tensor(5, synth.W, synth.POW2W, 0, (B, 1, H), bf16=False)
+    q = synth.tensor(5, synth.Q, synth.NORMAL, 0, (B, 1, 2, 8))
+    kv = synth.tensor(5, synth.KV, synth.NORMAL, 0, (B, Lk, 8))
+    layers = [dict(q_idx=qi, k_idx=ki, w=w, q=q, kv=kv)]
+    idx, out, _, _ = oracle_mod.indexcache_forward(
+        "F", layers, B=B, Lq=1, Lk=Lk, start_pos=Lk, H=H, dI=dI, k=64, n_h=2, Dqk=8, Dv=8,
+        scale=0.3)
+    assert idx[0, 0, 0].tolist() == list(range(Lk)) + [-1] * (64 - Lk)
+    o, _ = oracle_mod.dense_attn_row(q[0, 0], kv[0], kv[0], Lk, 0.3)
+    np.testing.assert_allclose(out[0, 0, 0], o, rtol=1e-13, atol=1e-15)

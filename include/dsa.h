@@ -1,0 +1,155 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) library for DeepSeek Sparse Attention
+ * (DSA) layer stacks under IndexCache.
+ *
+ * Sources.  [IC] "读懂 IndexCache：从 DSA 的选词开销到跨层索引复用" (the
+ * IndexCache explainer): §1.1 (F and S layers; the first layer must be F),
+ * §1.2 and its Figure 2 loop (the index cache is set on F layers, read on S
+ * layers; every layer attends with its own Q/K/V), §1.2's cost note (indexer
+ * work O(N L^2) -> O(M L^2)).  [IDX] "注意力机制中的 Index：从位置下标到预算
+ * 检索": §1 (visible set P_t = {s : 0 <= s < t}), §2 (sparse softmax over the
+ * selected set S_t), §4 (lightning indexer score, TopK over s < t, MLA latent
+ * rows shared by all query heads), §6.5 (top-k must be deterministic).
+ *
+ * Conventions shared by every entry point.
+ *  - bf16 tensors are raw IEEE bfloat16 bit patterns (dsa_bf16); all tensors
+ *    are dense, row-major, in DEVICE memory unless stated otherwise, and must
+ *    be 16-byte aligned.
+ *  - Query row i of a sequence sits at absolute position t = start_pos + i and
+ *    may see key positions s < t (t <= Lk is required).  Prefill: start_pos =
+ *    0, Lq = Lk.  Decode: Lq = 1, start_pos = Lk.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream), allocates nothing and never synchronises.  The caller
+ *    owns every buffer, including the workspace and the index cache.
+ *  - Argument errors are reported before anything is enqueued.  A kernel whose
+ *    bounded internal wait expires records it in a device error word and
+ *    returns early; dsa_check_device_errors() reports it as DSA_ERR_TIMEOUT.
+ *  - Results are deterministic: the same inputs give bit-identical indices
+ *    and outputs on every run ([IDX] §6.5).
+ *  - The library is not re-entrant across host threads for dsa_last_error().
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t dsa_bf16;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment */
+  DSA_ERR_BAD_PATTERN = 2, /* pattern empty, not 'F'/'S', or pattern[0] != 'F' */
+  DSA_ERR_UNSUPPORTED = 3, /* shape outside what the kernels implement */
+  DSA_ERR_WORKSPACE = 4,   /* ws_bytes below the *_workspace() requirement */
+  DSA_ERR_CUDA = 5,        /* a CUDA runtime/driver call or launch failed */
+  DSA_ERR_TIMEOUT = 6      /* a kernel's bounded wait expired (device word) */
+} dsa_status;
+
+/* Human-readable description of the most recent non-OK status. */
+const char *dsa_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Lightning indexer + top-k (F layers).  [IDX] §4: for each query row t,
+ *   I[t,s] = sum_{j<H_I} w[t,j] * ReLU(q_idx[t,j,:] . k_idx[s,:]),  s < t,
+ *   S_t = TopK_k { I[t,s] }.
+ * Output row idx[b,i,:] lists the selected positions in ascending order,
+ * followed by -1 padding when fewer than k positions are visible; equal
+ * scores prefer the lower position (-0.0 equals +0.0).  Scores are formed in
+ * fp32 from bf16 products (exact for integer-valued inputs and power-of-two
+ * weights).  The L x L score matrix is never written.  Scale factors such as
+ * d_I^-1/2 or H_I^-1/2 are folded into w by the caller (ReLU(c x) = c ReLU(x)
+ * for c > 0).
+ *   q_idx [B, Lq, H_I, d_I] bf16;  k_idx [B, Lk, d_I] bf16;  w [B, Lq, H_I] f32
+ *   idx   [B, Lq, k] int32 (written)
+ * Supported: H_I in {4, 8, 16, 32, 64}; d_I in {32, 64, 128}; 1 <= k <= 4096;
+ * B >= 1; Lq >= 1; start_pos >= 0; start_pos + Lq - 1 <= Lk.
+ * Workspace: dsa_indexer_topk_workspace() bytes, contents undefined on entry. */
+size_t dsa_indexer_topk_workspace(int B, int Lq, int Lk, int start_pos, int H_I,
+                                  int d_I, int k);
+dsa_status dsa_indexer_topk(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
+                            const float *w, int B, int Lq, int Lk, int start_pos,
+                            int H_I, int d_I, int k, int32_t *idx, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Sparse core attention.  [IDX] §2: for each query row t and head h,
+ *   e_r   = scale * q[t,h,:] . K[S_t[r], 0:D_qk]      (valid r: S_t[r] >= 0)
+ *   out[t,h,:] = sum_r softmax_r(e) * V[S_t[r], 0:D_v]
+ *   lse[t,h]   = log sum_r exp(e_r)  (natural log; -inf for an empty set)
+ * An empty set gives out = 0.  MLA ([IDX] §4): pass k = v = the latent cache
+ * with row stride 576, D_qk = 576, D_v = 512 (V is the first 512 columns);
+ * every query head reads the same latent row.  Index rows come from
+ * dsa_indexer_topk (any order is accepted; -1 entries are skipped; valid
+ * entries must satisfy 0 <= S_t[r] < t).
+ *   q   [B, Lq, n_h, D_qk] bf16
+ *   kbuf rows: kbuf + (b*Lk + s)*k_row_stride, D_qk bf16 each
+ *   vbuf rows: vbuf + (b*Lk + s)*v_row_stride, D_v bf16 each
+ *   idx [B, Lq, k] int32;  out [B, Lq, n_h, D_v] bf16 (written)
+ *   lse [B, Lq, n_h] f32 (written; may be NULL)
+ * Supported: (n_h, D_qk, D_v) = (128, 576, 512) or n_h <= 128 with
+ * D_qk, D_v in {64, 128}; 1 <= k <= 4096; row strides multiples of 8.
+ * Workspace: dsa_sparse_attn_workspace() bytes. */
+size_t dsa_sparse_attn_workspace(int B, int Lq, int n_h, int D_v, int k);
+dsa_status dsa_sparse_attn(const dsa_bf16 *q, const dsa_bf16 *kbuf,
+                           int64_t k_row_stride, const dsa_bf16 *vbuf,
+                           int64_t v_row_stride, const int32_t *idx, int B,
+                           int Lq, int Lk, int start_pos, int n_h, int D_qk,
+                           int D_v, int k, float scale, dsa_bf16 *out,
+                           float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * The IndexCache layer loop.  [IC] §1.1-§1.2, Figure 2:
+ *   for each layer l: if pattern[l] == 'F': idx_cache = TopK(indexer_l)
+ *                     out_l = sparse_attention_l(q_l, K_l, V_l, idx_cache)
+ * S layers launch no indexer work and read idx_cache in place: no copy and
+ * no memory beyond the single caller-owned idx_cache [B, Lq, k] int32.  On
+ * return (stream order) idx_cache holds the last F layer's indices.
+ * Projections, normalisation and the FFN between layers are outside this
+ * library; each layer's tensors are given directly in `layers`.
+ * pattern: n_layers characters 'F' or 'S' (no terminator needed), first 'F'.
+ * For S layers q_idx/k_idx/w are ignored and may be NULL.
+ * Workspace: indexcache_forward_workspace() bytes (shared by all layers). */
+typedef struct {
+  int B, Lq, Lk, start_pos; /* batch and positions, as above */
+  int H_I, d_I, k;          /* indexer heads, head dim, top-k budget */
+  int n_h, D_qk, D_v;       /* main attention heads and dims */
+  float scale;              /* main-attention logit scale */
+  int64_t k_row_stride, v_row_stride; /* element strides of K / V rows */
+} dsa_dims;
+
+typedef struct {
+  const dsa_bf16 *q_idx; /* [B, Lq, H_I, d_I]   F layers only */
+  const dsa_bf16 *k_idx; /* [B, Lk, d_I]        F layers only */
+  const float *w;        /* [B, Lq, H_I]        F layers only */
+  const dsa_bf16 *q;     /* [B, Lq, n_h, D_qk] */
+  const dsa_bf16 *kbuf;  /* K rows (see dsa_sparse_attn) */
+  const dsa_bf16 *vbuf;  /* V rows; == kbuf for MLA */
+  dsa_bf16 *out;         /* [B, Lq, n_h, D_v] */
+  float *lse;            /* [B, Lq, n_h] or NULL */
+} dsa_layer_io;
+
+size_t indexcache_forward_workspace(const dsa_dims *dims);
+dsa_status indexcache_forward(const char *pattern, int n_layers,
+                              const dsa_layer_io *layers, const dsa_dims *dims,
+                              int32_t *idx_cache, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/* Number of dsa_indexer_topk launches issued by this process so far (host
+ * counter; lets callers check that S layers run no indexer work). */
+long long dsa_indexer_launch_count(void);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns DSA_ERR_TIMEOUT if any kernel's bounded wait expired since the last
+ * call, DSA_ERR_CUDA on a CUDA error, DSA_OK otherwise. */
+dsa_status dsa_check_device_errors(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,230 @@
+// dsa_api.cu -- the C ABI (include/dsa.h): argument validation, workspace
+// sizing, the IndexCache layer loop and error reporting.  All compute runs in
+// the kernels of indexer_topk.cu and sparse_attn.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "dsa_internal.h"
+#include "dsa_ptx.cuh"
+
+namespace dsa {
+
+__device__ unsigned int g_dsa_error = 0;
+
+namespace {
+std::string g_last_error = "no error";
+std::atomic<long long> g_indexer_launches{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+dsa_status set_error(dsa_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+unsigned int* device_error_word() {
+  static unsigned int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dsa_error) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<unsigned int*>(p);
+  }
+  return cache[dev];
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+namespace {
+
+dsa_status check_indexer_args(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
+                              int B, int Lq, int Lk, int start_pos, int H, int d, int k,
+                              const int32_t* idx) {
+  if (!q_idx || !k_idx || !w || !idx)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_indexer_topk: null pointer");
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(idx))
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_indexer_topk: pointers must be 16-byte aligned");
+  if (B < 1 || Lq < 1 || Lk < 1 || start_pos < 0 || k < 1)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_indexer_topk: sizes must be positive");
+  if (static_cast<long long>(start_pos) + Lq - 1 > Lk)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_indexer_topk: start_pos + Lq - 1 exceeds Lk");
+  if (!indexer_supported(H, d, k))
+    return set_error(DSA_ERR_UNSUPPORTED,
+                     "dsa_indexer_topk: need H_I in {4,8,16,32,64}, d_I in {32,64,128}, k <= 2048");
+  if (static_cast<long long>(Lq) * H > (1ll << 31) - 1 || static_cast<long long>(B) * Lq * k > (1ll << 40))
+    return set_error(DSA_ERR_UNSUPPORTED, "dsa_indexer_topk: tensor too large");
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_last_error(void) { return g_last_error.c_str(); }
+
+long long dsa_indexer_launch_count(void) { return g_indexer_launches.load(); }
+
+size_t dsa_indexer_topk_workspace(int B, int Lq, int Lk, int start_pos, int H_I, int d_I, int k) {
+  (void)H_I;
+  (void)d_I;
+  if (B < 1 || Lq < 1 || k < 1 || start_pos < 0) return 0;
+  return indexer_plan(B, Lq, Lk, start_pos, std::min(k, 2048)).total_bytes;
+}
+
+dsa_status dsa_indexer_topk(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w, int B,
+                            int Lq, int Lk, int start_pos, int H_I, int d_I, int k, int32_t* idx,
+                            void* ws, size_t ws_bytes, void* stream) {
+  dsa_status st = check_indexer_args(q_idx, k_idx, w, B, Lq, Lk, start_pos, H_I, d_I, k, idx);
+  if (st != DSA_OK) return st;
+  if (!ws || !aligned16(ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_indexer_topk: null or misaligned workspace");
+  st = indexer_topk_launch(q_idx, k_idx, w, B, Lq, Lk, start_pos, H_I, d_I, k, idx, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
+  if (st == DSA_OK) g_indexer_launches.fetch_add(1);
+  return st;
+}
+
+size_t dsa_sparse_attn_workspace(int B, int Lq, int n_h, int D_v, int k) {
+  if (B < 1 || Lq < 1 || n_h < 1 || D_v < 1 || k < 1) return 0;
+  return sparse_attn_ws_bytes(B, Lq, n_h, D_v, k);
+}
+
+dsa_status dsa_sparse_attn(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
+                           const dsa_bf16* vbuf, int64_t v_row_stride, const int32_t* idx, int B,
+                           int Lq, int Lk, int start_pos, int n_h, int D_qk, int D_v, int k,
+                           float scale, dsa_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (!q || !kbuf || !vbuf || !idx || !out)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn: null pointer");
+  if (!aligned16(q) || !aligned16(kbuf) || !aligned16(vbuf) || !aligned16(idx) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn: pointers must be 16-byte aligned");
+  if (B < 1 || Lq < 1 || Lk < 1 || start_pos < 0 || n_h < 1 || D_qk < 1 || D_v < 1 || k < 1)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn: sizes must be positive");
+  if (static_cast<long long>(start_pos) + Lq - 1 > Lk)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn: start_pos + Lq - 1 exceeds Lk");
+  if (k_row_stride < D_qk || v_row_stride < D_v || (k_row_stride % 8) || (v_row_stride % 8))
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn: row strides must cover the row and be multiples of 8");
+  return sparse_attn_launch(q, kbuf, k_row_stride, vbuf, v_row_stride, idx, B, Lq, Lk, start_pos,
+                            n_h, D_qk, D_v, k, scale, out, lse, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));
+}
+
+size_t indexcache_forward_workspace(const dsa_dims* d) {
+  if (!d) return 0;
+  return std::max(dsa_indexer_topk_workspace(d->B, d->Lq, d->Lk, d->start_pos, d->H_I, d->d_I, d->k),
+                  dsa_sparse_attn_workspace(d->B, d->Lq, d->n_h, d->D_v, d->k));
+}
+
+dsa_status indexcache_forward(const char* pattern, int n_layers, const dsa_layer_io* layers,
+                              const dsa_dims* dims, int32_t* idx_cache, void* ws, size_t ws_bytes,
+                              void* stream) {
+  // [IC] §1.1: layer roles are F (own indexer) or S (reuse); the first layer
+  // must be F so that S layers always find an index tensor.
+  if (!pattern || n_layers < 1) return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward: empty pattern");
+  if (pattern[0] != 'F')
+    return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward: the first layer must be 'F'");
+  for (int l = 0; l < n_layers; ++l)
+    if (pattern[l] != 'F' && pattern[l] != 'S')
+      return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward: pattern entries must be 'F' or 'S'");
+  if (!layers || !dims || !idx_cache)
+    return set_error(DSA_ERR_INVALID_ARG, "indexcache_forward: null pointer");
+  const dsa_dims& d = *dims;
+  if (ws_bytes < indexcache_forward_workspace(dims))
+    return set_error(DSA_ERR_WORKSPACE, "indexcache_forward: workspace too small");
+  // Validate every layer before enqueueing anything.
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_layer_io& L = layers[l];
+    if (pattern[l] == 'F') {
+      dsa_status st = check_indexer_args(L.q_idx, L.k_idx, L.w, d.B, d.Lq, d.Lk, d.start_pos,
+                                         d.H_I, d.d_I, d.k, idx_cache);
+      if (st != DSA_OK) return st;
+    }
+    if (!L.q || !L.kbuf || !L.vbuf || !L.out)
+      return set_error(DSA_ERR_INVALID_ARG, "indexcache_forward: null attention pointer");
+  }
+  // [IC] §1.2, Figure 2: F layers refresh the cache, every layer attends
+  // with its own q/K/V through the cached positions.
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_layer_io& L = layers[l];
+    if (pattern[l] == 'F') {
+      dsa_status st = dsa_indexer_topk(L.q_idx, L.k_idx, L.w, d.B, d.Lq, d.Lk, d.start_pos, d.H_I,
+                                       d.d_I, d.k, idx_cache, ws, ws_bytes, stream);
+      if (st != DSA_OK) return st;
+    }
+    dsa_status st = dsa_sparse_attn(L.q, L.kbuf, d.k_row_stride, L.vbuf, d.v_row_stride, idx_cache,
+                                    d.B, d.Lq, d.Lk, d.start_pos, d.n_h, d.D_qk, d.D_v, d.k,
+                                    d.scale, L.out, L.lse, ws, ws_bytes, stream);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_check_device_errors(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("stream sync: ") + cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_dsa_error, sizeof(word));
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("read error word: ") + cudaGetErrorString(e));
+  if (word) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_dsa_error, &zero, sizeof(zero));
+    return set_error(DSA_ERR_TIMEOUT, "a kernel's bounded wait expired");
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// dsa_internal.h -- host-side helpers shared by the library's translation
+// units (not part of the public C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// Records a message for dsa_last_error() and returns `st`.
+dsa_status set_error(dsa_status st, const std::string& msg);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
+// link dependency).  Returns false on failure.
+bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle swizzle);
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
+// Device address of the library's error word on the current device.
+unsigned int* device_error_word();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- indexer + top-k (indexer_topk.cu)
+struct IndexerPlan {
+  int S;           // key splits per query block
+  int split_len;   // keys per split (multiple of 128)
+  int n_qblocks;   // query blocks of 8 rows per sequence
+  int n_items;     // B * n_qblocks * S
+  int grid;        // persistent CTAs
+  int cap;         // candidate-buffer capacity per query slot (entries)
+  size_t cand_bytes, split_bytes, split_cnt_bytes, total_bytes;
+};
+bool indexer_supported(int H, int d, int k);
+IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k);
+dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
+                               int B, int Lq, int Lk, int start_pos, int H, int d, int k,
+                               int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+// ---- sparse attention (sparse_attn.cu)
+size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k);
+dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
+                              const dsa_bf16* vbuf, int64_t v_row_stride, const int32_t* idx,
+                              int B, int Lq, int Lk, int start_pos, int n_h, int D_qk, int D_v,
+                              int k, float scale, dsa_bf16* out, float* lse, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
+
+}  // namespace dsa

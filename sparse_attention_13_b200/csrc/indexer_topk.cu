@@ -1,0 +1,770 @@
+// indexer_topk.cu -- fused lightning indexer + streaming exact top-k (sm_100a).
+//
+// Computes, for every query row t, I[t,s] = sum_j w[t,j] ReLU(q[t,j].k[s]) over
+// the visible keys s < t and keeps the k best positions ("注意力机制中的 Index",
+// §4: index-score equation and TopK over s < t; ties go to the lower position,
+// output ascending with -1 padding).  The L x L score matrix never exists.
+//
+// Design (one persistent CTA per SM, 320 threads):
+//   warp 8   TMA producer: the 8-query block of q (resident, [8*H, d] bf16) and
+//            a ring of 128-key tiles of k_idx, both 128B/64B-swizzled.
+//   warp 9   UMMA issuer: per key tile and query half (4 queries) one
+//            128 x (4H) x d MMA chain, D = keys x (query, head) in TMEM fp32,
+//            double-buffered (2 x 256 columns).  Keys sit on the M side so each
+//            TMEM lane is one key and the ReLU/head-weighted sum over the
+//            4H columns of a query needs no cross-lane reduction.
+//   warps 0-7 epilogue: tcgen05.ld a key's H head dots per query, fold
+//            w[t,j]*max(dot,0) in fp32 (fixed head order -> deterministic),
+//            pack (order-preserving score key << 32 | ~s) into one uint64 so a
+//            plain integer order is (score desc, position asc), and append the
+//            entries that beat the query's running threshold to a per-query
+//            candidate buffer, in ascending s.  When a buffer passes 2k entries
+//            an exact radix select (8-bit digits, in registers) keeps the best k
+//            in place (stable) and raises the threshold to the k-th value.  At
+//            the end of the block a final select writes the row.
+// Long rows in tiny grids (decode) split the key range across CTAs; each
+// split keeps its own top-k and a merge kernel selects the final k.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdio>
+
+#include "dsa_internal.h"
+#include "dsa_ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kQB = 8;        // queries per work item
+constexpr int kTileK = 128;   // keys per tile = UMMA M
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kEpiBar = 1;
+constexpr int kMaxK = 2048;
+constexpr int kSelRows = (2 * kMaxK + kTileK + kEpiThreads - 1) / kEpiThreads;  // 17
+constexpr int kMaxGrid = 160;
+constexpr int kTmemCols = 512;
+constexpr int kSmemBudget = 227 * 1024;
+
+__host__ __device__ constexpr int cap_for(int k) { return 2 * k + kTileK; }
+
+template <int H, int D>
+struct Cfg {
+  static constexpr int kChunkElems = D < 64 ? D : 64;
+  static constexpr int kChunkBytes = kChunkElems * 2;
+  static constexpr int kChunks = D / kChunkElems;
+  static constexpr uint32_t kSwz = kChunkBytes == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr int kSBO = 8 * kChunkBytes;
+  static constexpr int kHalfRows = 4 * H;                        // q rows of 4 queries
+  static constexpr int kQHalfBytes = kHalfRows * kChunkBytes;    // one (chunk, half) block
+  static constexpr int kQBytes = kQB * H * D * 2;
+  static constexpr int kKeyChunkBytes = kTileK * kChunkBytes;
+  static constexpr int kStageBytes = kTileK * D * 2;
+  static constexpr int kFixed = kQBytes + kQB * H * 4 + 8192;    // q + w + small state
+  static constexpr int kStagesFit = (kSmemBudget - 1024 - kFixed) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
+  static_assert(kStages >= 2, "shared memory too small for two key stages");
+  static_assert(kHalfRows <= 256, "TMA box rows");
+  static_assert(kQHalfBytes % 512 == 0, "swizzle atom alignment");
+};
+
+struct SelShared {
+  int hist[256];
+  int wcnt[kSelRows][kEpiWarps];
+  int woff[kSelRows][kEpiWarps];
+  int sel_bin, kk_new, bin_count, total;
+  unsigned long long minval;
+};
+
+struct EpiShared {
+  unsigned long long thr[kQB];
+  int cnt[2][kQB];
+  int qcount[2][kQB][4];
+  SelShared sel;
+};
+
+struct Params {
+  const float* w;        // [B, Lq, H]
+  int32_t* idx;          // [B, Lq, k]
+  uint64_t* cand;        // [grid][kQB][cap]
+  uint64_t* split_out;   // [B*Lq][S][k]
+  int* split_cnt;        // [B*Lq][S]
+  unsigned int* err;     // device error word
+  int B, Lq, Lk, start_pos, k, cap;
+  int S, split_len, n_qblocks, n_items;
+};
+
+struct Item {
+  int b, qb, split;
+  int s_begin, s_end;   // key range [s_begin, s_end) scanned by this item
+  int n_tiles;
+  int nq[2];            // valid queries per half
+};
+
+__device__ __forceinline__ Item decode_item(const Params& p, int w) {
+  Item it;
+  it.split = w % p.S;
+  const int rest = w / p.S;
+  it.b = rest % p.B;
+  it.qb = p.n_qblocks - 1 - rest / p.B;  // longest query blocks first
+  const int i0 = it.qb * kQB;
+  const int nvalid = min(kQB, p.Lq - i0);
+  it.nq[0] = max(0, min(4, nvalid));
+  it.nq[1] = max(0, min(4, nvalid - 4));
+  const int t_max = p.start_pos + i0 + nvalid - 1;  // largest visible count in the block
+  it.s_begin = it.split * p.split_len;
+  it.s_end = min(t_max, it.s_begin + p.split_len);
+  it.n_tiles = it.s_end > it.s_begin ? (it.s_end - it.s_begin + kTileK - 1) / kTileK : 0;
+  return it;
+}
+
+// Item sequence of a CTA: snake order over rounds of `grid` items.
+__device__ __forceinline__ int item_of(int round, int cta, int grid) {
+  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ unsigned long long pack_entry(float score, int s) {
+  return (static_cast<unsigned long long>(float_key(score)) << 32) |
+         static_cast<unsigned long long>(~static_cast<uint32_t>(s));
+}
+
+// ------------------------------------------------------------------ select
+// Exact top-k of buf[0, cnt) (distinct uint64 entries in ascending-s order)
+// by all 256 epilogue threads.  mode 0: keep the best k in place (stable),
+// return the k-th largest value.  mode 1: write the selected positions to
+// out_idx (ascending) and pad with -1 up to k.  mode 2: copy the selected
+// entries to out_list and their number to *out_count.
+__device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inplace,
+                                          int cnt, int k, int mode, int32_t* out_idx,
+                                          uint64_t* out_list, int* out_count, SelShared& sh) {
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  unsigned long long v[kSelRows];
+#pragma unroll
+  for (int r = 0; r < kSelRows; ++r) {
+    const int e = r * kEpiThreads + tid;
+    v[r] = e < cnt ? src[e] : 0ull;
+  }
+  unsigned long long thr = 0ull;  // keep entries >= thr
+  if (cnt > k) {
+    unsigned long long prefix = 0ull;
+    int kk = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      sh.hist[tid] = 0;
+      named_bar_sync(kEpiBar, kEpiThreads);
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) {
+        const int e = r * kEpiThreads + tid;
+        if (e < cnt) {
+          const bool match = shift == 56 || ((v[r] >> (shift + 8)) == (prefix >> (shift + 8)));
+          if (match) atomicAdd(&sh.hist[(v[r] >> shift) & 255ull], 1);
+        }
+      }
+      named_bar_sync(kEpiBar, kEpiThreads);
+      if (warp == 0) {
+        int loc[8];
+        int s = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { loc[i] = sh.hist[lane * 8 + i]; s += loc[i]; }
+        int incl = s;  // inclusive suffix sum over lanes >= lane
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, incl, off);
+          if (lane + off < 32) incl += y;
+        }
+        int above = incl - s;  // entries in bins of higher lanes
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (above < kk && above + loc[i] >= kk) {
+            sh.sel_bin = lane * 8 + i;
+            sh.kk_new = kk - above;
+            sh.bin_count = loc[i];
+          }
+          above += loc[i];
+        }
+      }
+      named_bar_sync(kEpiBar, kEpiThreads);
+      const int bin = sh.sel_bin;
+      prefix |= static_cast<unsigned long long>(bin) << shift;
+      kk = sh.kk_new;
+      if (sh.bin_count == kk) break;
+    }
+    thr = prefix;
+  }
+  // stable compaction of entries >= thr, row-major over (r, warp, lane)
+  unsigned mask[kSelRows];
+#pragma unroll
+  for (int r = 0; r < kSelRows; ++r) {
+    const int e = r * kEpiThreads + tid;
+    const bool keep = e < cnt && v[r] >= thr;
+    mask[r] = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) sh.wcnt[r][warp] = __popc(mask[r]);
+  }
+  if (tid == 0) sh.minval = ~0ull;
+  named_bar_sync(kEpiBar, kEpiThreads);
+  if (warp == 0) {
+    constexpr int kN = kSelRows * kEpiWarps;
+    constexpr int kPer = (kN + 31) / 32;
+    int loc[kPer];
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      loc[i] = e < kN ? (&sh.wcnt[0][0])[e] : 0;
+      s += loc[i];
+    }
+    int incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int run = incl - s;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      if (e < kN) (&sh.woff[0][0])[e] = run;
+      run += loc[i];
+    }
+    if (lane == 31) sh.total = incl;
+  }
+  named_bar_sync(kEpiBar, kEpiThreads);
+  const int total = sh.total;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned long long local_min = ~0ull;
+#pragma unroll
+  for (int r = 0; r < kSelRows; ++r) {
+    if (mask[r] & (1u << lane)) {
+      const int pos = sh.woff[r][warp] + __popc(mask[r] & lt);
+      if (mode == 0) {
+        dst_inplace[pos] = v[r];
+        local_min = v[r] < local_min ? v[r] : local_min;
+      } else if (mode == 1) {
+        out_idx[pos] = static_cast<int32_t>(~static_cast<uint32_t>(v[r] & 0xffffffffull));
+      } else {
+        out_list[pos] = v[r];
+      }
+    }
+  }
+  unsigned long long result = 0ull;
+  if (mode == 0) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, local_min, off);
+      local_min = o < local_min ? o : local_min;
+    }
+    if (lane == 0) atomicMin(&sh.minval, local_min);
+    named_bar_sync(kEpiBar, kEpiThreads);
+    result = sh.minval;
+  } else if (mode == 1) {
+    for (int pos = total + tid; pos < k; pos += kEpiThreads) out_idx[pos] = -1;
+  } else {
+    if (tid == 0) *out_count = total;
+  }
+  named_bar_sync(kEpiBar, kEpiThreads);
+  return result;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int H, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const Params p) {
+  using C = Cfg<H, D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* q_smem = smem;
+  uint8_t* key_smem = q_smem + C::kQBytes;
+  float* w_smem = reinterpret_cast<float*>(key_smem + C::kStages * C::kStageBytes);
+  EpiShared* es = reinterpret_cast<EpiShared*>(w_smem + kQB * H);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(es + 1);
+  uint64_t* key_full = bars;
+  uint64_t* key_empty = bars + C::kStages;
+  uint64_t* tmem_full = bars + 2 * C::kStages;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* q_full = tmem_empty + 2;
+  uint64_t* q_empty = q_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* consumed_tiles = abort_flag + 1;  // key tiles retired by the MMA warp
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int grid = gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) { mbar_init(&key_full[s], 1); mbar_init(&key_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], kEpiWarps); }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    *abort_flag = 0;
+    *consumed_tiles = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  int issued_tiles = 0;  // producer lane 0 only
+  if (warp == kTmaWarp) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int n_items_done = 0;
+      for (int round = 0;; ++round) {
+        const int w = item_of(round, cta, grid);
+        if (round * grid >= p.n_items) break;
+        if (w >= p.n_items) continue;
+        const Item it = decode_item(p, w);
+        if (it.n_tiles == 0) continue;
+        if (!mbar_wait(q_empty, (n_items_done & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          for (int h = 0; h < 2; ++h)
+            tma_load_3d(q_smem + (c * 2 + h) * C::kQHalfBytes, &tm_q, q_full,
+                        c * C::kChunkElems, (it.qb * kQB + 4 * h) * H, it.b);
+        bool ok = true;
+        for (int j = 0; j < it.n_tiles; ++j) {
+          if (!mbar_wait(&key_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&key_full[stage], C::kStageBytes);
+          uint8_t* dst = key_smem + stage * C::kStageBytes;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(dst + c * C::kKeyChunkBytes, &tm_k, &key_full[stage],
+                        c * C::kChunkElems, it.s_begin + j * kTileK, it.b);
+          ++issued_tiles;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        ++n_items_done;
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------- UMMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t unit = 0;
+      int n_items_done = 0;
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int w = item_of(round, cta, grid);
+        if (round * grid >= p.n_items) break;
+        if (w >= p.n_items) continue;
+        const Item it = decode_item(p, w);
+        if (it.n_tiles == 0) continue;
+        if (!mbar_wait(q_full, n_items_done & 1, abort_flag)) break;
+        tc_fence_after();
+        for (int j = 0; j < it.n_tiles && ok; ++j) {
+          if (!mbar_wait(&key_full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(key_smem + stage * C::kStageBytes);
+          for (int h = 0; h < 2; ++h) {
+            if (it.nq[h] == 0) continue;
+            const uint32_t buf = unit & 1;
+            if (!mbar_wait(&tmem_empty[buf], ((unit >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const int n = ((it.nq[h] * H + 15) / 16) * 16;
+            const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
+            const uint32_t d_tmem = tmem_base + buf * 256;
+            const uint32_t b_base = smem_u32(q_smem) + h * C::kQHalfBytes;
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c) {
+#pragma unroll
+              for (int kk = 0; kk < C::kChunkElems / 16; ++kk) {
+                const uint64_t ad = make_smem_desc(a_base + c * C::kKeyChunkBytes + kk * 32, 16,
+                                                   C::kSBO, C::kSwz);
+                const uint64_t bd = make_smem_desc(b_base + c * 2 * C::kQHalfBytes + kk * 32, 16,
+                                                   C::kSBO, C::kSwz);
+                umma_bf16_ss(d_tmem, ad, bd, idesc, (c | kk) != 0);
+              }
+            }
+            umma_commit(&tmem_full[buf]);
+            ++unit;
+          }
+          umma_commit(&key_empty[stage]);
+          *consumed_tiles = *consumed_tiles + 1;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        umma_commit(q_empty);
+        ++n_items_done;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int qd = warp & 3;       // TMEM lane quadrant
+    const int jp = warp >> 2;      // query pair within a half
+    const int tid = threadIdx.x;
+    uint32_t unit = 0;
+    for (int round = 0;; ++round) {
+      const int w = item_of(round, cta, grid);
+      if (round * grid >= p.n_items) break;
+      if (w >= p.n_items) continue;
+      const Item it = decode_item(p, w);
+      const int i0 = it.qb * kQB;
+      // per-item state
+      if (tid < kQB) {
+        es->thr[tid] = 0ull;
+        es->cnt[0][tid] = 0;
+      }
+      for (int e = tid; e < kQB * H; e += kEpiThreads) {
+        const int qs = e / H;
+        const int i = i0 + qs;
+        w_smem[e] = i < p.Lq ? p.w[(static_cast<size_t>(it.b) * p.Lq + i) * H + (e % H)] : 0.f;
+      }
+      named_bar_sync(kEpiBar, kEpiThreads);
+      uint64_t* cand_base = p.cand + static_cast<size_t>(cta) * kQB * p.cap;
+      bool ok = true;
+      for (int j = 0; j < it.n_tiles && ok; ++j) {
+        const int par = j & 1;
+        const int s = it.s_begin + j * kTileK + qd * 32 + lane;
+        for (int h = 0; h < 2; ++h) {
+          if (it.nq[h] == 0) continue;
+          const uint32_t buf = unit & 1;
+          if (!mbar_wait(&tmem_full[buf], (unit >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          float acc[2];
+          const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + buf * 256;
+          if constexpr (H >= 32) {
+            uint32_t v[2][H];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+              for (int c = 0; c < H / 32; ++c)
+                tmem_ld32<32>(t_lane + (2 * jp + jj) * H + c * 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(&v[jj][c * 32]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const float4* w4 = reinterpret_cast<const float4*>(w_smem + (4 * h + 2 * jp + jj) * H);
+              float a = 0.f;
+#pragma unroll
+              for (int c = 0; c < H / 4; ++c) {
+                const float4 ww = w4[c];
+                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 0]), 0.f), ww.x, a);
+                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 1]), 0.f), ww.y, a);
+                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 2]), 0.f), ww.z, a);
+                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 3]), 0.f), ww.w, a);
+              }
+              acc[jj] = a;
+            }
+          } else {
+            uint32_t v[2][H];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+              tmem_ld32<H>(t_lane + (2 * jp + jj) * H, v[jj]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const float* wq = w_smem + (4 * h + 2 * jp + jj) * H;
+              float a = 0.f;
+#pragma unroll
+              for (int c = 0; c < H; ++c) a = fmaf(fmaxf(__uint_as_float(v[jj][c]), 0.f), wq[c], a);
+              acc[jj] = a;
+            }
+          }
+          // candidate test and ordered append
+          unsigned long long P[2];
+          unsigned msk[2];
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            const int qs = 4 * h + 2 * jp + jj;
+            const int i = i0 + qs;
+            const int T = p.start_pos + i;
+            const bool valid = (i < p.Lq) && (s < T) && (s < it.s_end);
+            P[jj] = pack_entry(acc[jj], s);
+            const bool cand = valid && P[jj] > es->thr[qs];
+            msk[jj] = __ballot_sync(0xffffffffu, cand);
+            if (lane == 0) es->qcount[par][qs][qd] = __popc(msk[jj]);
+          }
+          named_bar_sync(kEpiBar, kEpiThreads);
+          bool need_sel = false;
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            const int qs = 4 * h + 2 * jp + jj;
+            const int base = es->cnt[par][qs];
+            int off = base;
+            for (int x = 0; x < qd; ++x) off += es->qcount[par][qs][x];
+            if (msk[jj] & (1u << lane)) {
+              cand_base[static_cast<size_t>(qs) * p.cap + off + __popc(msk[jj] & ((1u << lane) - 1u))] = P[jj];
+            }
+          }
+          // every thread derives the new counts of the half's 4 queries
+          int newcnt[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int qs = 4 * h + q4;
+            newcnt[q4] = es->cnt[par][qs] + es->qcount[par][qs][0] + es->qcount[par][qs][1] +
+                         es->qcount[par][qs][2] + es->qcount[par][qs][3];
+            need_sel |= newcnt[q4] > p.cap - kTileK;
+          }
+          if (tid < 4) es->cnt[par ^ 1][4 * h + tid] = newcnt[tid];
+          if (need_sel) {
+            named_bar_sync(kEpiBar, kEpiThreads);  // appends and counts visible
+#pragma unroll 1
+            for (int q4 = 0; q4 < 4; ++q4) {
+              if (newcnt[q4] <= p.cap - kTileK) continue;
+              const int qs = 4 * h + q4;
+              uint64_t* bq = cand_base + static_cast<size_t>(qs) * p.cap;
+              const unsigned long long kth =
+                  select_topk(bq, bq, newcnt[q4], p.k, 0, nullptr, nullptr, nullptr, es->sel);
+              if (tid == 0) {
+                es->thr[qs] = kth;
+                es->cnt[par ^ 1][qs] = p.k;
+              }
+            }
+            named_bar_sync(kEpiBar, kEpiThreads);
+          }
+          ++unit;
+        }
+      }
+      if (!ok) break;
+      // final selection per query row
+      named_bar_sync(kEpiBar, kEpiThreads);
+      const int fpar = it.n_tiles & 1;
+#pragma unroll 1
+      for (int qs = 0; qs < kQB; ++qs) {
+        const int i = i0 + qs;
+        if (i >= p.Lq) break;
+        const int c = es->cnt[fpar][qs];
+        const uint64_t* bq = cand_base + static_cast<size_t>(qs) * p.cap;
+        const size_t row = static_cast<size_t>(it.b) * p.Lq + i;
+        if (p.S == 1) {
+          select_topk(bq, nullptr, c, p.k, 1, p.idx + row * p.k, nullptr, nullptr, es->sel);
+        } else {
+          const size_t slot = row * p.S + it.split;
+          select_topk(bq, nullptr, c, p.k, 2, nullptr, p.split_out + slot * p.k,
+                      p.split_cnt + slot, es->sel);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == kTmaWarp && lane == 0) {
+    // Abort path only: let key-tile loads that no MMA consumed land before
+    // the CTA's shared memory is released (bounded; a load that never lands
+    // leaves nothing more to do).
+    for (int t = *consumed_tiles; t < issued_tiles; ++t) {
+      const uint32_t a = smem_u32(&key_full[t % C::kStages]);
+      const uint32_t par = (t / C::kStages) & 1;
+      const long long t0 = clock64();
+      while (!mbar_try_wait(a, par) && clock64() - t0 < kWaitLimitCycles) {}
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, 1u);
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ merge
+// Final top-k over the S per-split candidate lists of one query row.
+// Concatenating the lists in split order keeps ascending positions, so a
+// stable filter yields the ascending output row directly.
+constexpr int kMergeThreads = 512;
+
+__global__ void __launch_bounds__(kMergeThreads)
+indexer_merge_kernel(const uint64_t* __restrict__ split_out, const int* __restrict__ split_cnt,
+                     int32_t* __restrict__ idx, int S, int k) {
+  __shared__ int off[33];
+  __shared__ int hist[256];
+  __shared__ int sel_bin, kk_new, bin_count;
+  __shared__ int scan[kMergeThreads];
+  const size_t row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const uint64_t* lists = split_out + row * S * k;
+  if (tid == 0) {
+    int acc = 0;
+    for (int j = 0; j < S; ++j) { off[j] = acc; acc += split_cnt[row * S + j]; }
+    off[S] = acc;
+  }
+  __syncthreads();
+  const int n = off[S];
+  auto at = [&](int e) -> unsigned long long {
+    int j = 0;
+    while (off[j + 1] <= e) ++j;
+    return lists[static_cast<size_t>(j) * k + (e - off[j])];
+  };
+  unsigned long long thr = 0ull;
+  if (n > k) {
+    unsigned long long prefix = 0ull;
+    int kk = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      if (tid < 256) hist[tid] = 0;
+      __syncthreads();
+      for (int e = tid; e < n; e += kMergeThreads) {
+        const unsigned long long v = at(e);
+        if (shift == 56 || (v >> (shift + 8)) == (prefix >> (shift + 8)))
+          atomicAdd(&hist[(v >> shift) & 255ull], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int above = 0;
+        for (int b = 255; b >= 0; --b) {
+          if (above < kk && above + hist[b] >= kk) {
+            sel_bin = b; kk_new = kk - above; bin_count = hist[b];
+            break;
+          }
+          above += hist[b];
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<unsigned long long>(sel_bin) << shift;
+      kk = kk_new;
+      const bool done = bin_count == kk;
+      __syncthreads();
+      if (done) break;
+    }
+    thr = prefix;
+  }
+  // stable compaction over contiguous segments
+  const int per = (n + kMergeThreads - 1) / kMergeThreads;
+  const int e0 = tid * per, e1 = min(n, e0 + per);
+  int c = 0;
+  for (int e = e0; e < e1; ++e) c += at(e) >= thr;
+  scan[tid] = c;
+  __syncthreads();
+  for (int d = 1; d < kMergeThreads; d <<= 1) {
+    const int y = tid >= d ? scan[tid - d] : 0;
+    __syncthreads();
+    scan[tid] += y;
+    __syncthreads();
+  }
+  int pos = scan[tid] - c;
+  const int total = scan[kMergeThreads - 1];
+  int32_t* out = idx + row * k;
+  for (int e = e0; e < e1; ++e) {
+    const unsigned long long v = at(e);
+    if (v >= thr) out[pos++] = static_cast<int32_t>(~static_cast<uint32_t>(v & 0xffffffffull));
+  }
+  for (int q = total + tid; q < k; q += kMergeThreads) out[q] = -1;
+}
+
+template <int H, int D>
+dsa_status launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const Params& p, int grid,
+                     cudaStream_t stream) {
+  using C = Cfg<H, D>;
+  // At least 120 KB so that one CTA owns each SM (and all of its TMEM).
+  const int smem = std::max(120 * 1024, 1024 + C::kQBytes + C::kStages * C::kStageBytes +
+                                            kQB * H * 4 + static_cast<int>(sizeof(EpiShared)) +
+                                            (2 * C::kStages + 6) * 8 + 32);
+  auto kern = indexer_topk_kernel<H, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer smem attribute: ") + cudaGetErrorString(e));
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer launch: ") + cudaGetErrorString(e));
+  return DSA_OK;
+}
+
+}  // namespace
+
+bool indexer_supported(int H, int d, int k) {
+  const bool h_ok = H == 4 || H == 8 || H == 16 || H == 32 || H == 64;
+  const bool d_ok = d == 32 || d == 64 || d == 128;
+  return h_ok && d_ok && k >= 1 && k <= kMaxK;
+}
+
+IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k) {
+  (void)Lk;
+  IndexerPlan pl{};
+  pl.n_qblocks = (Lq + kQB - 1) / kQB;
+  const int t_max = start_pos + Lq - 1;
+  const int max_tiles = t_max > 0 ? (t_max + kTileK - 1) / kTileK : 0;
+  const long long base_items = static_cast<long long>(B) * pl.n_qblocks;
+  int S = 1;
+  if (base_items < 148) {
+    S = static_cast<int>(148 / base_items);
+    S = std::min(S, std::max(1, max_tiles / 8));
+    S = std::min(S, 32);
+  }
+  pl.S = S;
+  const int tiles_per_split = max_tiles > 0 ? (max_tiles + S - 1) / S : 1;
+  pl.split_len = tiles_per_split * kTileK;
+  pl.n_items = static_cast<int>(base_items * S);
+  pl.grid = std::min(pl.n_items, kMaxGrid);
+  pl.cap = cap_for(k);
+  pl.cand_bytes = static_cast<size_t>(kMaxGrid) * kQB * pl.cap * 8;
+  const size_t rows = static_cast<size_t>(B) * Lq;
+  pl.split_bytes = S > 1 ? rows * S * k * 8 : 0;
+  pl.split_cnt_bytes = S > 1 ? ((rows * S * 4 + 255) / 256) * 256 : 0;
+  pl.total_bytes = pl.cand_bytes + pl.split_bytes + pl.split_cnt_bytes;
+  return pl;
+}
+
+dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
+                               int B, int Lq, int Lk, int start_pos, int H, int d, int k,
+                               int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  IndexerPlan pl = indexer_plan(B, Lq, Lk, start_pos, k);
+  if (ws_bytes < pl.total_bytes) return set_error(DSA_ERR_WORKSPACE, "indexer workspace too small");
+  const int sms = device_sm_count();
+  if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
+  const int grid = std::max(1, std::min(pl.grid, sms));
+
+  const int chunk = d < 64 ? d : 64;
+  const CUtensorMapSwizzle swz = chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap tq, tk;
+  if (!encode_tiled_3d(&tq, q_idx, d, static_cast<uint64_t>(Lq) * H, B, static_cast<uint64_t>(d) * 2,
+                       static_cast<uint64_t>(Lq) * H * d * 2, chunk, 4 * H, swz))
+    return set_error(DSA_ERR_CUDA, "tensor map for q_idx failed");
+  if (!encode_tiled_3d(&tk, k_idx, d, Lk, B, static_cast<uint64_t>(d) * 2,
+                       static_cast<uint64_t>(Lk) * d * 2, chunk, kTileK, swz))
+    return set_error(DSA_ERR_CUDA, "tensor map for k_idx failed");
+
+  Params p{};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p.w = w;
+  p.idx = idx;
+  p.cand = reinterpret_cast<uint64_t*>(base);
+  p.split_out = pl.S > 1 ? reinterpret_cast<uint64_t*>(base + pl.cand_bytes) : nullptr;
+  p.split_cnt = pl.S > 1 ? reinterpret_cast<int*>(base + pl.cand_bytes + pl.split_bytes) : nullptr;
+  p.err = device_error_word();
+  if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k; p.cap = pl.cap;
+  p.S = pl.S; p.split_len = pl.split_len; p.n_qblocks = pl.n_qblocks; p.n_items = pl.n_items;
+
+  dsa_status st = DSA_ERR_UNSUPPORTED;
+#define DSA_CASE(HH, DD) \
+  if (H == HH && d == DD) st = launch_hd<HH, DD>(tq, tk, p, grid, stream);
+  DSA_CASE(4, 32) DSA_CASE(4, 64) DSA_CASE(4, 128)
+  DSA_CASE(8, 32) DSA_CASE(8, 64) DSA_CASE(8, 128)
+  DSA_CASE(16, 32) DSA_CASE(16, 64) DSA_CASE(16, 128)
+  DSA_CASE(32, 32) DSA_CASE(32, 64) DSA_CASE(32, 128)
+  DSA_CASE(64, 32) DSA_CASE(64, 64) DSA_CASE(64, 128)
+#undef DSA_CASE
+  if (st != DSA_OK) return st == DSA_ERR_UNSUPPORTED ? set_error(st, "indexer shape unsupported") : st;
+  if (pl.S > 1) {
+    indexer_merge_kernel<<<static_cast<unsigned>(static_cast<size_t>(B) * Lq), kMergeThreads, 0, stream>>>(
+        p.split_out, p.split_cnt, idx, pl.S, k);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge launch: ") + cudaGetErrorString(e));
+  }
+  return DSA_OK;
+}
+
+}  // namespace dsa

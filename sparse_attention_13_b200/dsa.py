@@ -1,0 +1,194 @@
+"""Python binding of the C ABI in include/dsa.h (argument marshalling only).
+
+Every function takes torch CUDA tensors, checks dtypes/shapes/contiguity,
+passes raw device pointers, sizes and the current stream to ``libdsa.so``
+and raises ``DSAError`` on a non-OK status.  All compute runs in the
+library's sm_100a kernels; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_BAD_PATTERN, DSA_ERR_UNSUPPORTED = 0, 1, 2, 3
+DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT = 4, 5, 6
+STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_BAD_PATTERN",
+                3: "DSA_ERR_UNSUPPORTED", 4: "DSA_ERR_WORKSPACE", 5: "DSA_ERR_CUDA",
+                6: "DSA_ERR_TIMEOUT"}
+
+EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
+           "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
+           "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors"]
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Lq", ctypes.c_int), ("Lk", ctypes.c_int),
+                ("start_pos", ctypes.c_int), ("H_I", ctypes.c_int), ("d_I", ctypes.c_int),
+                ("k", ctypes.c_int), ("n_h", ctypes.c_int), ("D_qk", ctypes.c_int),
+                ("D_v", ctypes.c_int), ("scale", ctypes.c_float),
+                ("k_row_stride", ctypes.c_int64), ("v_row_stride", ctypes.c_int64)]
+
+
+class LayerIO(ctypes.Structure):
+    _fields_ = [("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("q", ctypes.c_void_p), ("kbuf", ctypes.c_void_p), ("vbuf", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libdsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.dsa_last_error.restype = ctypes.c_char_p
+        L.dsa_indexer_topk_workspace.argtypes = [I] * 7
+        L.dsa_indexer_topk_workspace.restype = SZ
+        L.dsa_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, SZ, P]
+        L.dsa_indexer_topk.restype = I
+        L.dsa_sparse_attn_workspace.argtypes = [I] * 5
+        L.dsa_sparse_attn_workspace.restype = SZ
+        L.dsa_sparse_attn.argtypes = [P, P, I64, P, I64, P, I, I, I, I, I, I, I, I,
+                                      ctypes.c_float, P, P, P, SZ, P]
+        L.dsa_sparse_attn.restype = I
+        L.indexcache_forward_workspace.argtypes = [ctypes.POINTER(Dims)]
+        L.indexcache_forward_workspace.restype = SZ
+        L.indexcache_forward.argtypes = [ctypes.c_char_p, I, ctypes.POINTER(LayerIO),
+                                         ctypes.POINTER(Dims), P, P, SZ, P]
+        L.indexcache_forward.restype = I
+        L.dsa_indexer_launch_count.restype = ctypes.c_longlong
+        L.dsa_check_device_errors.argtypes = [P]
+        L.dsa_check_device_errors.restype = I
+        _lib = L
+    return _lib
+
+
+def _check(st: int) -> None:
+    if st != DSA_OK:
+        raise DSAError(st, lib().dsa_last_error().decode())
+
+
+def _stream(t=None):
+    import torch
+    dev = t.device if t is not None else None
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, shape=None, name="tensor"):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def indexer_topk_workspace(B, Lq, Lk, start_pos, H_I, d_I, k) -> int:
+    return int(lib().dsa_indexer_topk_workspace(B, Lq, Lk, start_pos, H_I, d_I, k))
+
+
+def indexer_topk(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None, ws=None):
+    """Lightning indexer + top-k.  q_idx [B,Lq,H,d] bf16, k_idx [B,Lk,d] bf16,
+    w [B,Lq,H] f32 -> idx [B,Lq,k] int32 (ascending positions, -1 padded)."""
+    import torch
+    B, Lq, H, d = q_idx.shape
+    Lk = k_idx.shape[1]
+    _need(q_idx, torch.bfloat16, name="q_idx")
+    _need(k_idx, torch.bfloat16, (B, Lk, d), "k_idx")
+    _need(w, torch.float32, (B, Lq, H), "w")
+    if out is None:
+        out = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device)
+    _need(out, torch.int32, (B, Lq, k), "out")
+    need = indexer_topk_workspace(B, Lq, Lk, start_pos, H, d, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_idx.device)
+    _check(lib().dsa_indexer_topk(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Lq, Lk, start_pos, H, d, k,
+                                  _ptr(out), _ptr(ws), ws.numel(), _stream(q_idx)))
+    return out
+
+
+def sparse_attn_workspace(B, Lq, n_h, D_v, k) -> int:
+    return int(lib().dsa_sparse_attn_workspace(B, Lq, n_h, D_v, k))
+
+
+def sparse_attn(q, kbuf, vbuf, idx, scale: float, *, D_v: int, start_pos: int = 0,
+                out=None, lse=None, ws=None):
+    """Sparse core attention.  q [B,Lq,n_h,D_qk] bf16; kbuf [B,Lk,Ck] and vbuf
+    [B,Lk,Cv] bf16 rows (K = first D_qk columns, V = first D_v columns; pass
+    the same latent tensor for MLA); idx [B,Lq,k] int32.
+    Returns out [B,Lq,n_h,D_v] bf16 (and fills ``lse`` [B,Lq,n_h] f32 if given)."""
+    import torch
+    B, Lq, n_h, D_qk = q.shape
+    Lk = kbuf.shape[1]
+    k = idx.shape[2]
+    _need(q, torch.bfloat16, name="q")
+    _need(kbuf, torch.bfloat16, name="kbuf")
+    _need(vbuf, torch.bfloat16, name="vbuf")
+    _need(idx, torch.int32, (B, Lq, k), "idx")
+    if out is None:
+        out = torch.empty((B, Lq, n_h, D_v), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (B, Lq, n_h, D_v), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (B, Lq, n_h), "lse")
+    need = sparse_attn_workspace(B, Lq, n_h, D_v, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().dsa_sparse_attn(_ptr(q), _ptr(kbuf), kbuf.shape[2], _ptr(vbuf), vbuf.shape[2],
+                                 _ptr(idx), B, Lq, Lk, start_pos, n_h, D_qk, D_v, k, scale,
+                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q)))
+    return out
+
+
+def make_dims(**kw) -> Dims:
+    return Dims(**kw)
+
+
+def indexcache_forward_workspace(dims: Dims) -> int:
+    return int(lib().indexcache_forward_workspace(ctypes.byref(dims)))
+
+
+def indexcache_forward(pattern: str, layers, dims: Dims, idx_cache, ws=None, stream=None):
+    """Runs the F/S layer loop.  ``layers`` is a list of dicts with keys
+    q_idx, k_idx, w (F layers), q, kbuf, vbuf, out and optionally lse."""
+    import torch
+    n = len(layers)
+    arr = (LayerIO * max(n, 1))()
+    for i, L in enumerate(layers):
+        arr[i] = LayerIO(*[L.get(f) and L[f].data_ptr() for f in
+                           ("q_idx", "k_idx", "w", "q", "kbuf", "vbuf", "out", "lse")])
+    need = indexcache_forward_workspace(dims)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=idx_cache.device)
+    st = stream if stream is not None else _stream(idx_cache)
+    _check(lib().indexcache_forward(pattern.encode(), n, arr, ctypes.byref(dims),
+                                    _ptr(idx_cache), _ptr(ws), ws.numel(), st))
+    return idx_cache
+
+
+def indexer_launch_count() -> int:
+    return int(lib().dsa_indexer_launch_count())
+
+
+def check_device_errors(stream=None) -> None:
+    _check(lib().dsa_check_device_errors(stream if stream is not None else _stream()))

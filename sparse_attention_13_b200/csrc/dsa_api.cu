@@ -61,6 +61,21 @@ bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                     uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride1_bytes};
+  const cuuint32_t box[2] = {box0, box1};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 unsigned int* device_error_word() {
   static unsigned int* cache[64] = {nullptr};
   int dev = 0;

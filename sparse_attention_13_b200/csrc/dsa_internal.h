@@ -17,6 +17,9 @@ dsa_status set_error(dsa_status st, const std::string& msg);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
 // link dependency).  Returns false on failure.
+bool encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                     uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle swizzle);
 bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                      uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
                      CUtensorMapSwizzle swizzle);

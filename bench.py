@@ -1,0 +1,577 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA layer stack under IndexCache on B200.
+
+Metric (one JSON line on rank 0): prefill tokens/s of a 16-layer stack at
+L = 200,000 with one F layer in four (FSSS x 4), plus decode ms/step of a
+48-layer 1/4-F stack with 8 sequences at 200,000 cached tokens, both with
+k = 2048, 64 indexer heads of dim 128 and MLA attention (128 heads, 576-wide
+latent, 512 value columns).  Inputs are seeded synthetic tensors generated on
+the device; every input of the timed region is larger than L2 (126 MB), so no
+flush is needed.  A prefill step runs, per layer, the indexer (F layers) and
+the sparse attention through the C ABI with CUDA events between launches;
+the e2e figure runs the public indexcache_forward() with inputs copied from
+pinned host memory every step and the final output copied back.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
+Multi-GPU: launched by torchrun, one independent replica per rank (weak scaling;
+no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s and decode ms/step at 200K ctx, 1/4-F IndexCache stack"
+
+PREFILL = dict(B=1, L=200000, layers=16, ratio=4, H_I=64, d_I=128, k=2048, n_h=128, D_qk=576, D_v=512)
+DECODE = dict(B=8, ctx=200000, layers=48, ratio=4, H_I=64, d_I=128, k=2048, n_h=128, D_qk=576, D_v=512)
+SEED = 1234
+
+
+def pattern_of(layers, ratio):
+    return "".join("F" if l % ratio == 0 else "S" for l in range(layers))
+
+
+# ----------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if self.uuid and self.uuid not in parts[1]:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1400.0, "fallback"
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "sparse_attention_13_b200", "csrc", d["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != d["sha256_16"]:
+            return None
+    return d["bytes_per_launch"]
+
+
+def attn_units(Lq, start_pos, k, B=1):
+    # selected (t, r) pairs: min(t, k) per query row
+    if start_pos == 0:
+        n_short = min(Lq, k)
+        return B * (n_short * (n_short - 1) // 2 + max(0, Lq - n_short) * k)
+    return B * Lq * min(start_pos, k)
+
+
+def indexer_pairs(Lq, start_pos, B=1):
+    if start_pos == 0:
+        return B * Lq * (Lq - 1) // 2
+    return B * Lq * start_pos
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_dsa(args):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_attention_13_b200 import dsa, synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    dev = torch.device("cuda", local)
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    seed = SEED + 1000 * rank
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    result = {}
+    # ---------------------------------------------------------------- prefill
+    P = dict(PREFILL)
+    if args.seq:
+        P["L"] = args.seq
+    L, k, pat = P["L"], P["k"], pattern_of(P["layers"], P["ratio"])
+    nF = pat.count("F")
+    bf, f32 = torch.bfloat16, torch.float32
+    q_idx, k_idx, w = {}, {}, {}
+    for l, role in enumerate(pat):
+        if role == "F":
+            q_idx[l] = torch.empty((1, L, P["H_I"], P["d_I"]), dtype=bf, device=dev)
+            k_idx[l] = torch.empty((1, L, P["d_I"]), dtype=bf, device=dev)
+            w[l] = torch.empty((1, L, P["H_I"]), dtype=f32, device=dev)
+            synth.fill_cuda(q_idx[l], seed, synth.Q_IDX, synth.INT9, l)
+            synth.fill_cuda(k_idx[l], seed, synth.K_IDX, synth.INT9, l)
+            synth.fill_cuda(w[l], seed, synth.W, synth.POW2W, l)
+    kv = []
+    for l in range(len(pat)):
+        t = torch.empty((1, L, P["D_qk"]), dtype=bf, device=dev)
+        synth.fill_cuda(t, seed, synth.KV, synth.NORMAL, l, sigma=0.5)
+        kv.append(t)
+    q = torch.empty((1, L, P["n_h"], P["D_qk"]), dtype=bf, device=dev)
+    synth.fill_cuda(q, seed, synth.Q, synth.NORMAL, 0, sigma=0.5)
+    out = torch.empty((1, L, P["n_h"], P["D_v"]), dtype=bf, device=dev)
+    idx = torch.empty((1, L, k), dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(P["D_qk"])
+    dims = dsa.make_dims(B=1, Lq=L, Lk=L, start_pos=0, H_I=P["H_I"], d_I=P["d_I"], k=k,
+                         n_h=P["n_h"], D_qk=P["D_qk"], D_v=P["D_v"], scale=scale,
+                         k_row_stride=P["D_qk"], v_row_stride=P["D_qk"])
+    ws = torch.empty(dsa.indexcache_forward_workspace(dims), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_launch = [0]
+
+    def step(events=None):
+        for l, role in enumerate(pat):
+            if role == "F":
+                if events is not None:
+                    events["idx"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                    events["idx"][-1][0].record(stream)
+                dsa.indexer_topk(q_idx[l], k_idx[l], w[l], k, out=idx, ws=ws)
+                if events is not None:
+                    events["idx"][-1][1].record(stream)
+            if events is not None:
+                events["attn"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                events["attn"][-1][0].record(stream)
+            dsa.sparse_attn(q, kv[l], kv[l], idx, scale, D_v=P["D_v"], out=out, ws=ws)
+            if events is not None:
+                events["attn"][-1][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    dsa.check_device_errors()
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    ev = {"idx": [], "attn": []}
+    t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(ev)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    dsa.check_device_errors()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["idx"])
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["attn"])
+    tokens = L * world
+    a_units = attn_units(L, 0, k)
+    i_pairs = indexer_pairs(L, 0)
+    attn_flops = a_units * 2 * P["n_h"] * (P["D_qk"] + P["D_v"])
+    idx_flops = i_pairs * 2 * P["H_I"] * P["d_I"]
+    result["prefill"] = dict(
+        ms_per_step=ms, tokens_per_s=tokens / (ms / 1e3), idx_ms=idx_ms, attn_ms=attn_ms,
+        indexer_share=nF * idx_ms / (nF * idx_ms + len(pat) * attn_ms),
+        attn_tflops=attn_flops / attn_ms / 1e9, idx_tflops=idx_flops / idx_ms / 1e9,
+        attn_flops=attn_flops, idx_flops=idx_flops, clocks=clk,
+        launches=args.steps * (nF + len(pat)))
+
+    # e2e through the public API with host buffers
+    host_in = []
+    for l in sorted(q_idx):
+        host_in += [(q_idx[l], None), (k_idx[l], None), (w[l], None)]
+    host_in += [(t, None) for t in kv] + [(q, None)]
+    host_in = [(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True)) for d, _ in host_in]
+    for d, h in host_in:
+        h.copy_(d)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(d.numel() * d.element_size() for d, _ in host_in)
+    d2h = out.numel() * out.element_size()
+    layers = []
+    for l, role in enumerate(pat):
+        L_ = dict(q=q, kbuf=kv[l], vbuf=kv[l], out=out)
+        if role == "F":
+            L_.update(q_idx=q_idx[l], k_idx=k_idx[l], w=w[l])
+        layers.append(L_)
+
+    def e2e_step():
+        for d, h in host_in:
+            d.copy_(h, non_blocking=True)
+        dsa.indexcache_forward(pat, layers, dims, idx, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    dsa.check_device_errors()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    result["prefill"]["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del host_in, out_h, q_idx, k_idx, w, kv, q, out, idx, ws, layers
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- decode
+    D = dict(DECODE)
+    B, ctx, kd = D["B"], D["ctx"], D["k"]
+    dpat = pattern_of(D["layers"], D["ratio"])
+    dq_idx, dk_idx, dw, dq, dkv = {}, {}, {}, [], []
+    for l, role in enumerate(dpat):
+        if role == "F":
+            dq_idx[l] = torch.empty((B, 1, D["H_I"], D["d_I"]), dtype=bf, device=dev)
+            dk_idx[l] = torch.empty((B, ctx, D["d_I"]), dtype=bf, device=dev)
+            dw[l] = torch.empty((B, 1, D["H_I"]), dtype=f32, device=dev)
+            synth.fill_cuda(dq_idx[l], seed + 7, synth.Q_IDX, synth.INT9, l)
+            synth.fill_cuda(dk_idx[l], seed + 7, synth.K_IDX, synth.INT9, l)
+            synth.fill_cuda(dw[l], seed + 7, synth.W, synth.POW2W, l)
+        t = torch.empty((B, 1, D["n_h"], D["D_qk"]), dtype=bf, device=dev)
+        synth.fill_cuda(t, seed + 7, synth.Q, synth.NORMAL, l, sigma=0.5)
+        dq.append(t)
+        t = torch.empty((B, ctx, D["D_qk"]), dtype=bf, device=dev)
+        synth.fill_cuda(t, seed + 7, synth.KV, synth.NORMAL, l, sigma=0.5)
+        dkv.append(t)
+    dout = torch.empty((B, 1, D["n_h"], D["D_v"]), dtype=bf, device=dev)
+    didx = torch.empty((B, 1, kd), dtype=torch.int32, device=dev)
+    ddims = dsa.make_dims(B=B, Lq=1, Lk=ctx, start_pos=ctx, H_I=D["H_I"], d_I=D["d_I"], k=kd,
+                          n_h=D["n_h"], D_qk=D["D_qk"], D_v=D["D_v"], scale=scale,
+                          k_row_stride=D["D_qk"], v_row_stride=D["D_qk"])
+    dws = torch.empty(dsa.indexcache_forward_workspace(ddims), dtype=torch.uint8, device=dev)
+
+    def dstep(events=None):
+        for l, role in enumerate(dpat):
+            if role == "F":
+                if events is not None:
+                    events["idx"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                    events["idx"][-1][0].record(stream)
+                dsa.indexer_topk(dq_idx[l], dk_idx[l], dw[l], kd, start_pos=ctx, out=didx, ws=dws)
+                if events is not None:
+                    events["idx"][-1][1].record(stream)
+            if events is not None:
+                events["attn"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                events["attn"][-1][0].record(stream)
+            dsa.sparse_attn(dq[l], dkv[l], dkv[l], didx, scale, D_v=D["D_v"], start_pos=ctx,
+                            out=dout, ws=dws)
+            if events is not None:
+                events["attn"][-1][1].record(stream)
+
+    dsteps = max(args.steps, 10)
+    for _ in range(max(args.warmup, 3)):
+        dstep()
+    barrier()
+    torch.cuda.synchronize(dev)
+    dclocks = ClockSampler(uuid)
+    dclocks.start()
+    dev_ev = {"idx": [], "attn": []}
+    t0.record(stream)
+    for _ in range(dsteps):
+        dstep(dev_ev)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    dclk = dclocks.stop()
+    barrier()
+    dsa.check_device_errors()
+    dms = max_over_ranks(t0.elapsed_time(t1) / dsteps)
+    d_idx_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["idx"])
+    d_attn_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["attn"])
+    nFd = dpat.count("F")
+    idx_bytes = B * ctx * D["d_I"] * 2 + B * D["H_I"] * D["d_I"] * 2 + B * kd * 4
+    attn_bytes = B * kd * D["D_qk"] * 2 + B * D["n_h"] * (D["D_qk"] + D["D_v"]) * 2 + B * kd * 4
+    step_bytes = nFd * idx_bytes + len(dpat) * attn_bytes
+    # e2e: new query tokens in, final output out; caches stay resident
+    dlayers = []
+    hq = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in dq]
+    hqi = [(dq_idx[l], torch.empty(dq_idx[l].shape, dtype=bf, pin_memory=True)) for l in sorted(dq_idx)]
+    hw = [(dw[l], torch.empty(dw[l].shape, dtype=f32, pin_memory=True)) for l in sorted(dw)]
+    for d_, h_ in hq + hqi + hw:
+        h_.copy_(d_)
+    hout = torch.empty(dout.shape, dtype=bf, pin_memory=True)
+    for l, role in enumerate(dpat):
+        L_ = dict(q=dq[l], kbuf=dkv[l], vbuf=dkv[l], out=dout)
+        if role == "F":
+            L_.update(q_idx=dq_idx[l], k_idx=dk_idx[l], w=dw[l])
+        dlayers.append(L_)
+
+    def de2e_step():
+        for d_, h_ in hq + hqi + hw:
+            d_.copy_(h_, non_blocking=True)
+        dsa.indexcache_forward(dpat, dlayers, ddims, didx, ws=dws)
+        hout.copy_(dout, non_blocking=True)
+
+    for _ in range(3):
+        de2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    t0.record(stream)
+    for _ in range(dsteps):
+        de2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    de2e_ms = max_over_ranks(t0.elapsed_time(t1) / dsteps)
+    dh2d = sum(d_.numel() * d_.element_size() for d_, _ in hq + hqi + hw)
+    result["decode"] = dict(ms_per_step=dms, idx_ms=d_idx_ms, attn_ms=d_attn_ms,
+                            step_bytes=step_bytes, clocks=dclk,
+                            e2e={"value": de2e_ms, "unit": "ms/step", "h2d_bytes_per_step": dh2d,
+                                 "d2h_bytes_per_step": hout.numel() * 2})
+    n_merge = 1  # the split decode indexer launches a merge kernel after each F layer
+    result["decode"]["launches"] = dsteps * (nFd * (1 + n_merge) + len(dpat))
+    result["peaks"] = (hbm_peak, tc_peak, peak_kind)
+    result["world"] = world
+    if world > 1:
+        dist.destroy_process_group()
+    return result
+
+
+# ----------------------------------------------------------------- CPU oracle
+_ORACLE_KEYS = {}
+
+
+def _oracle_keys(seed, B, L, d):
+    # indexer keys of sequence 0, layer 0 (host copy for the oracle sample)
+    import numpy as np
+
+    from sparse_attention_13_b200 import synth
+    key = (seed, B, L, d)
+    if key not in _ORACLE_KEYS:
+        _ORACLE_KEYS[key] = synth.rows(seed, synth.K_IDX, synth.INT9, 0, (B, L, d), np.arange(L))
+    return _ORACLE_KEYS[key]
+
+
+def oracle_sample(budget_rows=4, decode=True):
+    """Times the CPU oracle (single thread, as it stands) on a bounded sample
+    of the prefill and decode workloads and extrapolates to the metric."""
+    import numpy as np
+
+    import oracle
+    from sparse_attention_13_b200 import synth
+
+    oracle.build()
+    P = PREFILL
+    L, k = P["L"], P["k"]
+    nF = pattern_of(P["layers"], P["ratio"]).count("F")
+    seed = SEED
+    k_h = _oracle_keys(seed, 1, L, P["d_I"])[None]
+    ts = [int(L * (2 * j + 1) / (2 * budget_rows)) for j in range(budget_rows)]
+    t_idx, t_attn = [], []
+    for t in ts:
+        qr = synth.rows(seed, synth.Q_IDX, synth.INT9, 0, (1, L, P["H_I"], P["d_I"]),
+                        np.arange(P["H_I"]) + t * P["H_I"])
+        wr = synth.rows(seed, synth.W, synth.POW2W, 0, (1, L, P["H_I"]), [t], bf16=False)[0]
+        a = time.perf_counter()
+        I = oracle.indexer_row(qr, k_h[0], wr, t)
+        sel = oracle.topk_row(I, t, k)
+        t_idx.append(time.perf_counter() - a)
+        valid = sel[sel >= 0]
+        rows_kv = synth.rows(seed, synth.KV, synth.NORMAL, 0, (1, L, P["D_qk"]), valid, sigma=0.5)
+        q_r = synth.rows(seed, synth.Q, synth.NORMAL, 0, (1, L, P["n_h"], P["D_qk"]),
+                         np.arange(P["n_h"]) + t * P["n_h"], sigma=0.5)
+        a = time.perf_counter()
+        oracle.sparse_attn_row(q_r, rows_kv, rows_kv, np.arange(len(valid), dtype=np.int32),
+                               1 / math.sqrt(P["D_qk"]), Dv=P["D_v"])
+        t_attn.append(time.perf_counter() - a)
+    # per token of the stack: nF indexer rows (work ~ t, sampled at mean t) + all layers' attention
+    per_tok = nF * statistics.mean(t_idx) + P["layers"] * statistics.mean(t_attn)
+    res = {"prefill_tokens_per_s": 1.0 / per_tok,
+           "sample": f"{budget_rows} indexer rows (t = {ts}) and {budget_rows} attention rows "
+                     f"(k = {k}) of the L = {L} stack, single-threaded, extrapolated by "
+                     f"rows x layers (indexer work is linear in t; mean of stratified t)",
+           "seconds": sum(t_idx) + sum(t_attn)}
+    if decode:
+        Dd = DECODE
+        ctx = Dd["ctx"]
+        kd_h = _oracle_keys(seed + 7, Dd["B"], ctx, Dd["d_I"])
+        qr = synth.rows(seed + 7, synth.Q_IDX, synth.INT9, 0, (Dd["B"], 1, Dd["H_I"], Dd["d_I"]),
+                        np.arange(Dd["H_I"]))
+        wr = synth.rows(seed + 7, synth.W, synth.POW2W, 0, (Dd["B"], 1, Dd["H_I"]), [0], bf16=False)[0]
+        a = time.perf_counter()
+        I = oracle.indexer_row(qr, kd_h, wr, ctx)
+        sel = oracle.topk_row(I, ctx, Dd["k"])
+        ti = time.perf_counter() - a
+        valid = sel[sel >= 0]
+        rows_kv = synth.rows(seed + 7, synth.KV, synth.NORMAL, 0, (Dd["B"], ctx, Dd["D_qk"]), valid, sigma=0.5)
+        q_r = synth.rows(seed + 7, synth.Q, synth.NORMAL, 0, (Dd["B"], 1, Dd["n_h"], Dd["D_qk"]),
+                         np.arange(Dd["n_h"]), sigma=0.5)
+        a = time.perf_counter()
+        oracle.sparse_attn_row(q_r, rows_kv, rows_kv, np.arange(len(valid), dtype=np.int32),
+                               1 / math.sqrt(Dd["D_qk"]), Dv=Dd["D_v"])
+        ta = time.perf_counter() - a
+        nFd = pattern_of(Dd["layers"], Dd["ratio"]).count("F")
+        res["decode_ms_per_step"] = 1e3 * Dd["B"] * (nFd * ti + Dd["layers"] * ta)
+        res["decode_sample"] = (f"1 indexer row over {ctx} keys and 1 attention row, sequence 0, "
+                                f"single-threaded, extrapolated x {Dd['B']} sequences x layers")
+        res["seconds"] += ti + ta
+    return res
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    P = PREFILL
+    # each step: a bounded sample (one stratified indexer row + one attention row)
+    for _ in range(args.warmup):
+        oracle_sample(budget_rows=1, decode=False)
+    vals = []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(oracle_sample(budget_rows=1, decode=False)["prefill_tokens_per_s"])
+    elapsed = time.perf_counter() - t_all
+    v = statistics.mean(vals)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"prefill L={P['L']}, 16 layers FSSS x4, k=2048 (CPU oracle sample)",
+                       "global_batch": 1, "seq_len": P["L"], "parallelism": "single host thread"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "per step: 1 indexer row at t = L/2 and 1 attention row, "
+                                       "extrapolated to the 16-layer stack"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--seq", type=int, default=0, help="override the prefill length (testing)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, _ = dist_env()
+    res = run_dsa(args)
+    if rank != 0:
+        return
+    hbm_peak, tc_peak, peak_kind = res["peaks"]
+    pf, dc = res["prefill"], res["decode"]
+    attn_tr = traffic_for("mla_sparse_attn")
+    idx_tr = traffic_for("indexer_topk")
+    line = {
+        "metric": METRIC, "value": pf["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill: B=1, L=200000, 16 layers FSSS x4 (1/4 F), H_I=64 d_I=128 "
+                               "k=2048, MLA 128 heads 576/512; decode: B=8, ctx 200000, 48 layers "
+                               "1/4 F", "global_batch": world, "seq_len": PREFILL["L"],
+                   "parallelism": f"dp{world} (independent replicas)",
+                   "l2": "inputs larger than L2 (126 MB) every step; no flush"},
+        "roofline": {"bound": "tensor", "kernel": "mla_sparse_attn", "achieved": pf["attn_tflops"],
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": pf["attn_tflops"] / tc_peak,
+                     "traffic": attn_tr, "peak_kind": f"{peak_kind} bf16 sustained",
+                     "per_launch_flops": pf["attn_flops"], "avg_launch_ms": pf["attn_ms"]},
+        "roofline_indexer": {"bound": "tensor", "kernel": "indexer_topk", "achieved": pf["idx_tflops"],
+                             "peak": tc_peak, "unit": "TFLOP/s", "frac": pf["idx_tflops"] / tc_peak,
+                             "traffic": idx_tr, "per_launch_flops": pf["idx_flops"],
+                             "avg_launch_ms": pf["idx_ms"]},
+        "indexer_share": pf["indexer_share"],
+        "decode": {"ms_per_step": dc["ms_per_step"], "higher_is_better": False,
+                   "idx_launch_ms": dc["idx_ms"], "attn_launch_ms": dc["attn_ms"],
+                   "roofline": {"bound": "hbm", "achieved": dc["step_bytes"] / dc["ms_per_step"] / 1e6,
+                                "peak": hbm_peak, "unit": "GB/s",
+                                "frac": dc["step_bytes"] / dc["ms_per_step"] / 1e6 / hbm_peak,
+                                "traffic": None, "per_step_bytes": dc["step_bytes"]},
+                   "e2e": dc["e2e"], "clocks": dc["clocks"]},
+        "e2e": pf["e2e"],
+        "gpu_launches": pf["launches"],
+        "clocks": pf["clocks"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample()
+        line["cpu_baseline"] = {"value": cb["prefill_tokens_per_s"], "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle", "sample": cb["sample"],
+                                "decode_ms_per_step": cb["decode_ms_per_step"],
+                                "decode_sample": cb["decode_sample"]}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

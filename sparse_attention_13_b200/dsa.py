@@ -175,7 +175,7 @@ def indexcache_forward(pattern: str, layers, dims: Dims, idx_cache, ws=None, str
     n = len(layers)
     arr = (LayerIO * max(n, 1))()
     for i, L in enumerate(layers):
-        arr[i] = LayerIO(*[L.get(f) and L[f].data_ptr() for f in
+        arr[i] = LayerIO(*[(L[f].data_ptr() if L.get(f) is not None else None) for f in
                            ("q_idx", "k_idx", "w", "q", "kbuf", "vbuf", "out", "lse")])
     need = indexcache_forward_workspace(dims)
     if ws is None:

@@ -1,0 +1,113 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point of include/dsa.h, and rejects bad arguments on the host before any
+CUDA call (pattern rule of the IndexCache explainer §1.1: the first layer
+must be F).  CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_13_b200 import dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_]+)\s*\(", src)) - {"if", "sizeof"})
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dsa.lib()
+    names = _declared()
+    assert "indexcache_forward" in names and "dsa_indexer_topk" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(dsa.EXPORTS) <= set(names)
+
+
+def _fwd(pattern, n_layers=None, layers=None, dims=None, idx=1, ws=None, ws_bytes=0):
+    lib = dsa.lib()
+    n = len(pattern) if n_layers is None else n_layers
+    arr = layers if layers is not None else (dsa.LayerIO * max(n, 1))()
+    d = dims if dims is not None else dsa.Dims(B=1, Lq=8, Lk=8, start_pos=0, H_I=64, d_I=128, k=4,
+                                              n_h=128, D_qk=576, D_v=512, scale=1.0,
+                                              k_row_stride=576, v_row_stride=576)
+    return lib.indexcache_forward(pattern.encode(), n, arr, ctypes.byref(d),
+                                  ctypes.c_void_p(idx), ctypes.c_void_p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("pattern", ["SFFF", "S", "FXSS", "fsss", "FF S"])
+def test_bad_pattern_rejected(pattern):
+    assert _fwd(pattern) == dsa.DSA_ERR_BAD_PATTERN
+    assert dsa.lib().dsa_last_error()
+
+
+def test_empty_pattern_rejected():
+    assert _fwd("", n_layers=0) == dsa.DSA_ERR_BAD_PATTERN
+
+
+def test_null_pointers_rejected_before_launch():
+    # valid pattern, layer pointers all NULL
+    d = dsa.Dims(B=1, Lq=8, Lk=8, start_pos=0, H_I=64, d_I=128, k=4, n_h=128, D_qk=576, D_v=512,
+                 scale=1.0, k_row_stride=576, v_row_stride=576)
+    need = dsa.lib().indexcache_forward_workspace(ctypes.byref(d))
+    st = _fwd("FS", dims=d, ws=4096, ws_bytes=need)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_small_workspace_rejected():
+    d = dsa.Dims(B=1, Lq=64, Lk=64, start_pos=0, H_I=64, d_I=128, k=16, n_h=128, D_qk=576, D_v=512,
+                 scale=1.0, k_row_stride=576, v_row_stride=576)
+    assert _fwd("FS", dims=d, ws=4096, ws_bytes=16) == dsa.DSA_ERR_WORKSPACE
+
+
+def test_indexer_argument_checks():
+    lib = dsa.lib()
+    P = ctypes.c_void_p
+    a = P(1 << 20)  # aligned, never dereferenced: the checks fail first
+    # unsupported head count
+    st = lib.dsa_indexer_topk(a, a, a, 1, 8, 8, 0, 12, 128, 4, a, a, 1 << 30, None)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    # k too large for the kernel
+    st = lib.dsa_indexer_topk(a, a, a, 1, 8, 8, 0, 64, 128, 4096, a, a, 1 << 30, None)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    # query rows beyond the cache
+    st = lib.dsa_indexer_topk(a, a, a, 1, 8, 8, 5, 64, 128, 4, a, a, 1 << 30, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    # misaligned pointer
+    st = lib.dsa_indexer_topk(P((1 << 20) + 2), a, a, 1, 8, 8, 0, 64, 128, 4, a, a, 1 << 30, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    # null output
+    st = lib.dsa_indexer_topk(a, a, a, 1, 8, 8, 0, 64, 128, 4, None, a, 1 << 30, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_attention_argument_checks():
+    lib = dsa.lib()
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    # unsupported head dims (not MLA, too wide for the small-dim kernel)
+    st = lib.dsa_sparse_attn(a, a, 256, a, 256, a, 1, 8, 8, 0, 16, 256, 256, 4, 1.0, a, None, a,
+                             1 << 20, None)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    # row stride shorter than the row
+    st = lib.dsa_sparse_attn(a, a, 64, a, 576, a, 1, 8, 8, 0, 128, 576, 512, 4, 1.0, a, None, a,
+                             1 << 20, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes():
+    lib = dsa.lib()
+    small = lib.dsa_indexer_topk_workspace(1, 512, 512, 0, 4, 32, 64)
+    big = lib.dsa_indexer_topk_workspace(1, 200000, 200000, 0, 64, 128, 2048)
+    dec = lib.dsa_indexer_topk_workspace(8, 1, 200000, 200000, 64, 128, 2048)
+    assert 0 < small < big
+    assert dec > 0
+    assert lib.dsa_indexer_topk_workspace(0, 1, 1, 0, 64, 128, 4) == 0
+
+
+def test_launch_counter_starts_at_zero_without_launches():
+    assert dsa.indexer_launch_count() >= 0

@@ -66,7 +66,7 @@ const char *dsa_last_error(void);
  * for c > 0).
  *   q_idx [B, Lq, H_I, d_I] bf16;  k_idx [B, Lk, d_I] bf16;  w [B, Lq, H_I] f32
  *   idx   [B, Lq, k] int32 (written)
- * Supported: H_I in {4, 8, 16, 32, 64}; d_I in {32, 64, 128}; 1 <= k <= 4096;
+ * Supported: H_I in {4, 8, 16, 32, 64}; d_I in {32, 64, 128}; 1 <= k <= 2048;
  * B >= 1; Lq >= 1; start_pos >= 0; start_pos + Lq - 1 <= Lk.
  * Workspace: dsa_indexer_topk_workspace() bytes, contents undefined on entry. */
 size_t dsa_indexer_topk_workspace(int B, int Lq, int Lk, int start_pos, int H_I,
@@ -91,8 +91,9 @@ dsa_status dsa_indexer_topk(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
  *   vbuf rows: vbuf + (b*Lk + s)*v_row_stride, D_v bf16 each
  *   idx [B, Lq, k] int32;  out [B, Lq, n_h, D_v] bf16 (written)
  *   lse [B, Lq, n_h] f32 (written; may be NULL)
- * Supported: (n_h, D_qk, D_v) = (128, 576, 512) or n_h <= 128 with
- * D_qk, D_v in {64, 128}; 1 <= k <= 4096; row strides multiples of 8.
+ * Supported: (n_h, D_qk, D_v) = (128, 576, 512) with kbuf == vbuf, or
+ * n_h <= 128 with D_qk, D_v <= 128; k >= 1; row strides multiples of 8.
+ * Rows are read up to min(t, k) entries: valid entries first, -1 after.
  * Workspace: dsa_sparse_attn_workspace() bytes. */
 size_t dsa_sparse_attn_workspace(int B, int Lq, int n_h, int D_v, int k);
 dsa_status dsa_sparse_attn(const dsa_bf16 *q, const dsa_bf16 *kbuf,

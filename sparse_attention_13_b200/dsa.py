@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_BAD_PATTERN",
 
 EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
-           "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors"]
+           "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
+           "dsa_indexer_topk_noalloc"]
 
 
 class DSAError(RuntimeError):
@@ -71,6 +72,8 @@ def lib():
                                          ctypes.POINTER(Dims), P, P, SZ, P]
         L.indexcache_forward.restype = I
         L.dsa_indexer_launch_count.restype = ctypes.c_longlong
+        L.dsa_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P]
+        L.dsa_indexer_topk_noalloc.restype = I
         L.dsa_check_device_errors.argtypes = [P]
         L.dsa_check_device_errors.restype = I
         _lib = L
@@ -125,6 +128,27 @@ def indexer_topk(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None, ws=No
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_idx.device)
     _check(lib().dsa_indexer_topk(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Lq, Lk, start_pos, H, d, k,
                                   _ptr(out), _ptr(ws), ws.numel(), _stream(q_idx)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
+
+
+def indexer_topk_noalloc(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None):
+    """Same as indexer_topk, for callers that cannot hand the library a
+    workspace: the scratch comes from a fixed 48 MiB device array inside the
+    library (shared by every call; do not overlap calls on the GPU)."""
+    import torch
+    B, Lq, H, d = q_idx.shape
+    Lk = k_idx.shape[1]
+    _need(q_idx, torch.bfloat16, name="q_idx")
+    _need(k_idx, torch.bfloat16, (B, Lk, d), "k_idx")
+    _need(w, torch.float32, (B, Lq, H), "w")
+    if out is None:
+        out = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device)
+    _need(out, torch.int32, (B, Lq, k), "out")
+    _check(lib().dsa_indexer_topk_noalloc(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Lq, Lk, start_pos,
+                                          H, d, k, _ptr(out), _stream(q_idx)))
     return out
 
 

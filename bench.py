@@ -512,6 +512,52 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def kernel_case(name, seq, reps):
+    """Runs one kernel on a small case (inputs of a few GB, larger than L2) for
+    profiling: `reps` launches after one warm-up launch."""
+    import torch
+
+    from sparse_attention_13_b200 import dsa, synth
+    dev = torch.device("cuda", 0)
+    bf = torch.bfloat16
+    if name in ("indexer", "decode_idx"):
+        B, Lq, Lk, sp = (1, seq, seq, 0) if name == "indexer" else (8, 1, 200000, 200000)
+        q = torch.empty((B, Lq, 64, 128), dtype=bf, device=dev)
+        kk = torch.empty((B, Lk, 128), dtype=bf, device=dev)
+        w = torch.empty((B, Lq, 64), dtype=torch.float32, device=dev)
+        synth.fill_cuda(q, SEED, synth.Q_IDX, synth.INT9, 0)
+        synth.fill_cuda(kk, SEED, synth.K_IDX, synth.INT9, 0)
+        synth.fill_cuda(w, SEED, synth.W, synth.POW2W, 0)
+        out = torch.empty((B, Lq, 2048), dtype=torch.int32, device=dev)
+        ws = torch.empty(dsa.indexer_topk_workspace(B, Lq, Lk, sp, 64, 128, 2048), dtype=torch.uint8, device=dev)
+        run = lambda: dsa.indexer_topk(q, kk, w, 2048, start_pos=sp, out=out, ws=ws)
+    elif name in ("attn", "decode_attn"):
+        B, Lq, Lk, sp = (1, seq, seq, 0) if name == "attn" else (8, 1, 200000, 200000)
+        q = torch.empty((B, Lq, 128, 576), dtype=bf, device=dev)
+        kv = torch.empty((B, Lk, 576), dtype=bf, device=dev)
+        synth.fill_cuda(q, SEED, synth.Q, synth.NORMAL, 0, sigma=0.5)
+        synth.fill_cuda(kv, SEED, synth.KV, synth.NORMAL, 0, sigma=0.5)
+        # every row selects min(t, k) distinct positions below t (strided pattern)
+        r = torch.arange(2048, device=dev, dtype=torch.int64)[None, :]
+        t = torch.arange(Lq, device=dev, dtype=torch.int64)[:, None] + sp
+        pos = (r * 7919) % t.clamp(min=1)
+        idx = torch.where(r < t, pos, torch.full_like(pos, -1)).to(torch.int32)[None].expand(B, Lq, 2048).contiguous()
+        out = torch.empty((B, Lq, 128, 512), dtype=bf, device=dev)
+        run = lambda: dsa.sparse_attn(q, kv, kv, idx, 1 / math.sqrt(576), D_v=512, start_pos=sp, out=out)
+    else:
+        raise SystemExit(f"unknown kernel case {name}")
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    dsa.check_device_errors()
+    print(f"{name} seq={seq}: {e0.elapsed_time(e1) / reps:.3f} ms/launch", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,7 +566,12 @@ def main():
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--seq", type=int, default=0, help="override the prefill length (testing)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", default="", help="profiling: indexer|attn|decode_idx|decode_attn")
+    ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
+    if args.kernel_case:
+        kernel_case(args.kernel_case, args.seq or 16384, args.reps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

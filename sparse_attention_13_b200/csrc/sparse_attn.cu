@@ -6,24 +6,28 @@
 // columns).
 //
 // mla_sparse_attn_kernel (n_h = 128, D_qk = 576, D_v = 512, K = V = latent):
-//   A cluster of two CTAs owns one query row at a time.  CTA c holds half of
-//   the query in TMEM (Q[:, 288c : 288c+288], the A operand of the QK UMMA) and
-//   half of the output accumulator (O[:, 256c : 256c+256], fp32 in TMEM).
-//   Per chunk of 64 selected rows:
-//     producer warp  TMA gather4 of the chunk's latent rows, 5 slabs of 64
-//                    columns each (CTA0 columns 0..319, CTA1 256..575),
-//                    128B-swizzled, into a 3-stage ring;
-//     MMA warp       S_c = Q_c K_c^T over the CTA's 288 columns (18 K16 UMMAs,
-//                    A from TMEM), then, one chunk behind, O_c += P V_c with
-//                    V_c the gathered slabs read as an MN-major B operand;
-//     softmax warps  (thread = head = TMEM lane) read S_c, swap partial score
-//                    tiles with the peer CTA through distributed shared memory
-//                    (S = S_0 + S_1, identical in both CTAs because fp32
-//                    addition commutes), mask padded rows, run the online
-//                    softmax in the log2 domain with lazy rescaling of O
-//                    (only when the running max grows by more than 2^8), and
-//                    write P as bf16 into a double-buffered K-major tile.
+//   A cluster of two CTAs owns one query row (or one key-range split of it)
+//   at a time.  CTA0 holds latent columns 0..255 of the query in TMEM, CTA1
+//   columns 256..575 (the A operand of the QK UMMA); CTA c accumulates output
+//   columns 256c..256c+255 in TMEM (fp32).  Per chunk of 64 selected rows:
+//     4 producer warps  cp.async gather of the chunk's latent rows (CTA0: 4
+//                    slabs of 64 columns, CTA1: 5 slabs) into the 128B-swizzled
+//                    layout, 3-stage ring; each selected row is read from
+//                    memory exactly once;
+//     MMA warp       S_c = Q_c K_c^T over the CTA's columns (A from TMEM),
+//                    then, one chunk behind, O_c += P V_c with V_c the
+//                    gathered slabs 0..3 read as an MN-major B operand;
+//     8 softmax warps (thread = head = TMEM lane x half of the chunk) read
+//                    S_c, send the partial scores to the peer with st.async
+//                    (tx-counted on the peer's mbarrier, no fences), add the
+//                    peer's partial (S = S_0 + S_1, identical in both CTAs as
+//                    fp32 addition commutes), mask padded rows, run the online
+//                    softmax in the log2 domain with lazy rescaling of O (only
+//                    when the running max grows by more than 2^8), and write
+//                    P as bf16 into a double-buffered K-major tile.
 //   The finished row is normalised by the softmax sum and stored as bf16.
+//   Few long rows (decode) split the index list across clusters; the
+//   partials (normalised O and log-sum-exp) are combined by mla_merge_kernel.
 //
 // simt_sparse_attn_kernel: plain CUDA-core kernel for small head dims
 // (D_qk, D_v <= 128, separate K and V tensors), one block per query row.
@@ -99,56 +103,78 @@ simt_sparse_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
 // ------------------------------------------------------------------ MLA
 constexpr int kNH = 128, kDQK = 576, kDV = 512;
 constexpr int kChunk = 64;                     // selected rows per chunk (UMMA N of QK)
-constexpr int kSlabs = 5;                      // 64-column slabs gathered per CTA
-constexpr int kSlabBytes = kChunk * 128;       // 8 KB
-constexpr int kStageBytes = kSlabs * kSlabBytes;
+constexpr int kSlabBytes = kChunk * 128;       // one 64-column slab of a chunk, 8 KB
+constexpr int kMaxSlabs = 5;                   // CTA0: columns 0..255, CTA1: 256..575
+constexpr int kStageBytes = kMaxSlabs * kSlabBytes;
 constexpr int kStages = 3;
-constexpr int kPBytes = kNH * 128;             // P tile [128 heads][64 rows] bf16
 constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile fp32
-constexpr int kQSteps = 18;                    // 288 / 16
-constexpr uint32_t kOCol = 0, kSCol = 256, kQCol = 320;
-constexpr int kMlaThreads = 192;               // 4 softmax warps, producer, MMA
-constexpr int kProdWarp = 4, kMmaWarpA = 5;
+// TMEM columns: O (fp32, 256) | S (fp32, 64) | P (bf16 pairs, 32) | Q (bf16 pairs, 128 or 160)
+constexpr uint32_t kOCol = 0, kSCol = 256, kPCol = 320, kQCol = 352;
+constexpr int kSoftWarps = 8;
+constexpr int kProdWarp0 = 8, kProdWarps = 4, kMmaWarpA = 12;
+constexpr int kMlaThreads = 416;
 constexpr float kRescaleThresh = 8.0f;          // log2 units
+constexpr int kPairBarBase = 2;                 // named barriers 2..5: the two warps of a quadrant
 
 struct MlaBars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full, s_free;
   uint64_t p_full[2], pv_done[2];
   uint64_t o_full, o_free, q_full;
-  uint64_t x_full[2], x_free[2];
-  unsigned long long kvmask[kStages];
+  uint64_t x_full[2], xout_full, xout_free;
+  unsigned short kvmask[kStages][4];            // per producer warp: 16 rows each
+  float red[2][2][kNH];                         // [parity][half][head] chunk maxima
+  float lsum[2][2][kNH];                        // [kind][half][head] final sums
   uint32_t tmem_slot;
   int abort_flag;
 };
 
-constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 2 * kPBytes + 2 * kXBytes + 1024;
+// shared memory: gather ring | peer partials (double-buffered) | own partial staging
+constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 3 * kXBytes +
+                         static_cast<int>(sizeof(MlaBars)) + 64;
 
 struct MlaParams {
+  const __nv_bfloat16* kv;  // latent rows, row stride kv_stride
+  int64_t kv_stride;
   const __nv_bfloat16* q;   // [B*Lq][128][576]
   const int32_t* idx;       // [B*Lq][k]
   __nv_bfloat16* out;       // [B*Lq][128][512]
   float* lse;               // [B*Lq][128] or null
+  float* part_o;            // split partials [B*Lq][S][128][512] (S > 1)
+  float* part_lse;          // [B*Lq][S][128]
   unsigned int* err;
   int B, Lq, Lk, start_pos, k;
+  int S, cps;               // key-range splits per row, chunks per split
   float scale_log2;
 };
 
-__device__ __forceinline__ int item_chunks(const MlaParams& p, int item) {
-  const int i = item % p.Lq;
-  const int nv = min(p.start_pos + i, p.k);
-  return (nv + kChunk - 1) / kChunk;
+struct MlaItem {
+  int row, split, b, c0, n;  // chunks [c0, c0 + n) of the row's index list
+  int nv;                    // valid index entries read: min(t, k)
+};
+
+__device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int item) {
+  MlaItem it;
+  it.row = item / p.S;
+  it.split = item % p.S;
+  it.b = it.row / p.Lq;
+  const int i = it.row % p.Lq;
+  it.nv = min(p.start_pos + i, p.k);
+  const int nch = (it.nv + kChunk - 1) / kChunk;
+  it.c0 = it.split * p.cps;
+  it.n = max(0, min(nch, it.c0 + p.cps) - it.c0);
+  return it;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
-mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
+mla_sparse_attn_kernel(const MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* kv_smem = smem;
-  uint8_t* p_smem = kv_smem + kStages * kStageBytes;
-  uint8_t* x_smem = p_smem + 2 * kPBytes;
-  MlaBars* bb = reinterpret_cast<MlaBars*>(x_smem + 2 * kXBytes);
+  uint8_t* x_smem = kv_smem + kStages * kStageBytes;   // X_in[2]: the peer's partials
+  uint8_t* xo_smem = x_smem + 2 * kXBytes;             // X_out: this CTA's partial
+  MlaBars* bb = reinterpret_cast<MlaBars*>(xo_smem + kXBytes);
   volatile int* abort_flag = &bb->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,21 +182,32 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   const uint32_t peer = rank ^ 1u;
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
-  const int n_items = p.B * p.Lq;
+  const int n_items = p.B * p.Lq * p.S;
+  // CTA0 owns latent columns 0..255 (QK and V), CTA1 owns 256..575 (QK) and
+  // 256..511 (V); together they gather each selected row exactly once.
+  const int n_slabs = rank == 0 ? 4 : 5;
+  const int qk_steps = n_slabs * 4;
+  const int col0 = rank == 0 ? 0 : 256;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&bb->kv_full[s], 1); mbar_init(&bb->kv_empty[s], 1); }
-    mbar_init(&bb->s_full, 1);
-    mbar_init(&bb->s_free, 128);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bb->p_full[b], 128);
-      mbar_init(&bb->pv_done[b], 1);
-      mbar_init(&bb->x_full[b], 128);
-      mbar_init(&bb->x_free[b], 128);
+    // kv_full: one cp.async-completion arrival per producer thread plus one
+    // ordinary arrival per producer warp (after its validity mask is written)
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bb->kv_full[s], kProdWarps * 32 + kProdWarps);
+      mbar_init(&bb->kv_empty[s], 1);
     }
+    mbar_init(&bb->s_full, 1);
+    mbar_init(&bb->s_free, kSoftWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bb->p_full[b], kSoftWarps);
+      mbar_init(&bb->pv_done[b], 1);
+      mbar_init(&bb->x_full[b], 1);
+    }
+    mbar_init(&bb->xout_full, kSoftWarps);
+    mbar_init(&bb->xout_free, 1);
     mbar_init(&bb->o_full, 1);
-    mbar_init(&bb->o_free, 128);
-    mbar_init(&bb->q_full, 128);
+    mbar_init(&bb->o_free, kSoftWarps);
+    mbar_init(&bb->q_full, kSoftWarps);
     bb->abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,55 +215,59 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     tmem_alloc(&bb->tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp == kProdWarp && lane == 0) tma_prefetch_desc(&tm_kv);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bb->tmem_slot;
 
-  if (warp == kProdWarp) {
+  if (warp >= kProdWarp0 && warp < kProdWarp0 + kProdWarps) {
     // ------------------------------------------------------------ gather
+    // Producer warp pw copies rows 16pw..16pw+15 of each 64-row chunk: per
+    // row, consecutive lanes move consecutive 16-byte pieces of the CTA's
+    // columns into the 128B-swizzled slab layout the UMMAs read.
+    const int pw = warp - kProdWarp0;
+    const int n_pieces = n_slabs * 8;
     uint32_t g = 0;  // global chunk counter
     bool ok = true;
     for (int item = pair; item < n_items && ok; item += n_pairs) {
-      const int nch = item_chunks(p, item);
-      const int b = item / p.Lq;
-      const int i = item % p.Lq;
-      const int nv = min(p.start_pos + i, p.k);
-      const int32_t* irow = p.idx + static_cast<size_t>(item) * p.k;
-      for (int c = 0; c < nch; ++c, ++g) {
+      const MlaItem it = mla_item(p, item);
+      if (it.n == 0) continue;
+      const int32_t* irow = p.idx + static_cast<size_t>(it.row) * p.k;
+      const __nv_bfloat16* kvb = p.kv + static_cast<int64_t>(it.b) * p.Lk * p.kv_stride + col0;
+      auto fetch = [&](int c) -> int {
+        const int r = c * kChunk + pw * 16 + (lane & 15);
+        return (lane < 16 && r < it.nv) ? __ldg(irow + r) : -1;
+      };
+      int s_next = fetch(it.c0);
+      for (int c = it.c0; c < it.c0 + it.n; ++c, ++g) {
         const int stage = g % kStages;
         const uint32_t ph = (g / kStages) & 1;
+        const int sidx = s_next;
+        const bool valid = sidx >= 0 && sidx < p.Lk;
+        const int srow = valid ? sidx : 0;
+        const unsigned m = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+        if (c + 1 < it.c0 + it.n) s_next = fetch(c + 1);   // overlap the next chunk's index load
         if (!mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag)) { ok = false; break; }
-        const int r0 = c * kChunk + lane, r1 = r0 + 32;
-        const int s0 = r0 < nv ? irow[r0] : -1;
-        const int s1 = r1 < nv ? irow[r1] : -1;
-        const bool v0 = s0 >= 0 && s0 < p.Lk, v1 = s1 >= 0 && s1 < p.Lk;
-        const int row0 = b * p.Lk + (v0 ? s0 : 0);
-        const int row1 = b * p.Lk + (v1 ? s1 : 0);
-        const unsigned m0 = __ballot_sync(0xffffffffu, v0);
-        const unsigned m1 = __ballot_sync(0xffffffffu, v1);
-        if (lane == 0) {
-          bb->kvmask[stage] = static_cast<unsigned long long>(m0) | (static_cast<unsigned long long>(m1) << 32);
-          mbar_arrive_expect_tx(&bb->kv_full[stage], kStageBytes);
-        }
-        uint8_t* dst = kv_smem + stage * kStageBytes;
-        const int col0 = rank == 0 ? 0 : 256;
-#pragma unroll
-        for (int grp = 0; grp < 16; ++grp) {
-          const int src = (grp & 7) * 4;
-          const int a0 = __shfl_sync(0xffffffffu, grp < 8 ? row0 : row1, src + 0);
-          const int a1 = __shfl_sync(0xffffffffu, grp < 8 ? row0 : row1, src + 1);
-          const int a2 = __shfl_sync(0xffffffffu, grp < 8 ? row0 : row1, src + 2);
-          const int a3 = __shfl_sync(0xffffffffu, grp < 8 ? row0 : row1, src + 3);
-          if (lane == 0) {
-#pragma unroll
-            for (int sl = 0; sl < kSlabs; ++sl)
-              tma_gather4(dst + sl * kSlabBytes + grp * 512, &tm_kv, &bb->kv_full[stage],
-                          col0 + sl * 64, a0, a1, a2, a3);
+        const uint32_t dst = smem_u32(kv_smem + stage * kStageBytes);
+#pragma unroll 4
+        for (int rr = 0; rr < 16; ++rr) {
+          const int row_s = __shfl_sync(0xffffffffu, srow, rr);
+          const int r = pw * 16 + rr;
+          const __nv_bfloat16* src = kvb + static_cast<int64_t>(row_s) * p.kv_stride;
+          for (int piece = lane; piece < n_pieces; piece += 32) {
+            const int sl = piece >> 3, j = piece & 7;
+            cp_async_16(dst + sl * kSlabBytes + r * 128 + ((j ^ (r & 7)) << 4), src + piece * 8);
           }
         }
+        if (lane == 0) bb->kvmask[stage][pw] = static_cast<unsigned short>(m);
+        cp_async_arrive_noinc(&bb->kv_full[stage]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb->kv_full[stage]);
       }
+    }
+    if (!ok) {
+      // abort path: let this thread's copies land before the CTA can exit
+      asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else if (warp == kMmaWarpA) {
     // ------------------------------------------------------------ MMA
@@ -240,35 +281,31 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         if (!mbar_wait(&bb->p_full[pb], (gc >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const int stage = gc % kStages;
-        // V = this CTA's slabs 0..3: value columns 0..255 (CTA0) or 256..511 (CTA1)
+        // V = this CTA's slabs 0..3: value columns 0..255 (CTA0) or 256..511 (CTA1);
+        // A = P (bf16) in TMEM, 8 columns per 16 rows of the chunk
         const uint32_t v_base = smem_u32(kv_smem + stage * kStageBytes);
-        const uint32_t a_base = smem_u32(p_smem + pb * kPBytes);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t ad = make_smem_desc(a_base + kk * 32, 16, 1024, kSwizzle128B);
           const uint64_t bd = make_smem_desc(v_base + kk * 2048, kSlabBytes, 1024, kSwizzle128B);
-          umma_bf16_ss(tmem + kOCol, ad, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          umma_bf16_ts(tmem + kOCol, tmem + kPCol + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&bb->pv_done[pb]);
         umma_commit(&bb->kv_empty[stage]);
         return true;
       };
       for (int item = pair; item < n_items && ok; item += n_pairs) {
-        const int nch = item_chunks(p, item);
-        if (nch == 0) continue;
+        const MlaItem it = mla_item(p, item);
+        if (it.n == 0) continue;
         if (!mbar_wait(&bb->q_full, it_n & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int c = 0; c < nch && ok; ++c, ++g) {
+        for (int c = 0; c < it.n && ok; ++c, ++g) {
           const int stage = g % kStages;
           if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&bb->s_free, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kb = smem_u32(kv_smem + stage * kStageBytes);
-#pragma unroll
-          for (int st = 0; st < kQSteps; ++st) {
-            // CTA0: slabs 0..3 + first half of slab 4; CTA1: second half of slab 0 + slabs 1..4
-            const int e = rank == 0 ? st : st + 2;
-            const uint64_t bd = make_smem_desc(kb + (e >> 2) * kSlabBytes + (e & 3) * 32, 16, 1024,
+          for (int st = 0; st < qk_steps; ++st) {
+            const uint64_t bd = make_smem_desc(kb + (st >> 2) * kSlabBytes + (st & 3) * 32, 16, 1024,
                                                kSwizzle128B);
             umma_bf16_ts(tmem + kSCol, tmem + kQCol + st * 8, bd, idesc_qk, st != 0);
           }
@@ -279,117 +316,146 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           }
         }
         if (!ok) break;
-        if (nch == 1 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (!issue_pv(g - 1, nch == 1)) { ok = false; break; }
+        if (it.n == 1 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!issue_pv(g - 1, it.n == 1)) { ok = false; break; }
         umma_commit(&bb->o_full);
         ++it_n;
       }
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int h = threadIdx.x;  // head = TMEM lane
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t x_local = smem_u32(x_smem);
-    const uint32_t x_remote = mapa_shared(x_local, peer);
+    // thread = (head h = TMEM lane, half hf of the chunk's 64 columns)
+    const int qd = warp & 3, hf = warp >> 2;
+    const int h = qd * 32 + lane;
+    const int tid = threadIdx.x;
+    const int pair_bar = kPairBarBase + qd;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const uint32_t x_remote = mapa_shared(smem_u32(x_smem), peer);
     const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bb->x_full[0]), peer),
                                       mapa_shared(smem_u32(&bb->x_full[1]), peer)};
-    const uint32_t xfree_remote[2] = {mapa_shared(smem_u32(&bb->x_free[0]), peer),
-                                      mapa_shared(smem_u32(&bb->x_free[1]), peer)};
     uint32_t g = 0, it_n = 0;
     bool ok = true;
     for (int item = pair; item < n_items && ok; item += n_pairs) {
-      const int nch = item_chunks(p, item);
-      const size_t row = static_cast<size_t>(item);
-      __nv_bfloat16* orow = p.out + (row * kNH + h) * kDV + rank * 256;
-      if (nch == 0) {
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        for (int j = 0; j < 32; ++j) reinterpret_cast<uint4*>(orow)[j] = z;
-        if (p.lse && rank == 0) p.lse[row * kNH + h] = -INFINITY;
+      const MlaItem it = mla_item(p, item);
+      const bool partial = p.S > 1;
+      if (it.n == 0) {
+        if (partial) {
+          float* po = p.part_o + ((static_cast<size_t>(it.row) * p.S + it.split) * kNH + h) * kDV +
+                      rank * 256 + hf * 128;
+          for (int j = 0; j < 32; ++j) reinterpret_cast<float4*>(po)[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (rank == 0 && hf == 0)
+            p.part_lse[(static_cast<size_t>(it.row) * p.S + it.split) * kNH + h] = -INFINITY;
+        } else {
+          __nv_bfloat16* orow = p.out + (static_cast<size_t>(it.row) * kNH + h) * kDV + rank * 256 + hf * 128;
+          for (int j = 0; j < 16; ++j) reinterpret_cast<uint4*>(orow)[j] = make_uint4(0, 0, 0, 0);
+          if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = -INFINITY;
+        }
         continue;
       }
-      // this CTA's half of the query row -> TMEM (A operand of QK)
+      // this CTA's part of the query row -> TMEM (A operand of QK)
       {
-        const uint4* qsrc = reinterpret_cast<const uint4*>(p.q + (row * kNH + h) * kDQK + rank * 288);
-#pragma unroll
-        for (int blk = 0; blk < 5; ++blk) {
+        const uint4* qsrc = reinterpret_cast<const uint4*>(
+            p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0 + hf * 128);
+        const int nblk = hf == 0 ? 2 : (rank == 0 ? 2 : 3);
+        for (int blk = 0; blk < nblk; ++blk) {
           uint32_t r[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (blk * 8 + j < 36) v = __ldg(qsrc + blk * 8 + j);
+            const uint4 v = __ldg(qsrc + blk * 8 + j);
             r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
           }
-          tmem_st32x32(t_lane + kQCol + blk * 32, r);
+          tmem_st32x32(t_lane + kQCol + hf * 64 + blk * 32, r);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bb->q_full);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb->q_full);
       }
-      // l_run: sum of the bf16 weights that PV multiplies (normalises O);
-      // l_lse: the same sum in fp32 before rounding (for the log-sum-exp).
+      // l_run: sum of the bf16 weights PV multiplies (normalises O);
+      // l_lse: the same sum before rounding (for the log-sum-exp).  Each half
+      // of a head keeps the sums of its own columns.
       float m_run = -INFINITY, l_run = 0.f, l_lse = 0.f;
-      for (int c = 0; c < nch; ++c, ++g) {
+      for (int c = 0; c < it.n; ++c, ++g) {
         const int stage = g % kStages;
         const int xb = g & 1;
         if (!mbar_wait(&bb->s_full, g & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float s[64];
+        float s[32];
         {
           uint32_t v[32];
-          tmem_ld32<32>(t_lane + kSCol, v);
+          tmem_ld32<32>(t_lane + kSCol + hf * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
-          tmem_ld32<32>(t_lane + kSCol + 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
         }
         tc_fence_before();
-        mbar_arrive(&bb->s_free);
-        // swap partial scores with the peer: my partial -> peer's buffer xb
-        if (!mbar_wait_cluster(&bb->x_free[xb], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        {
-          const uint32_t rowbase = x_remote + xb * kXBytes + h * 256;
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            st_cluster_v4(rowbase + ((j ^ (h & 15)) << 4), s[4 * j], s[4 * j + 1], s[4 * j + 2],
-                          s[4 * j + 3]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb->s_free);
+        // Partial scores -> peer: stage them in X_out, one thread moves the
+        // whole 32 KB tile with a bulk DMA that completes on the peer's
+        // x_full[xb].  X_in is double-buffered; the peer can only send chunk
+        // g+2 after it received this CTA's chunk g+1, which is sent after
+        // X_in[xb] was consumed below, so no release handshake is needed.
+        if (tid == 0 && g > 0) {
+          bulk_wait_read_all();           // the previous DMA finished reading X_out
+          mbar_arrive(&bb->xout_free);
         }
-        mbar_arrive_remote(xfull_remote[xb]);
+        if (g > 0 && !mbar_wait(&bb->xout_free, (g - 1) & 1, abort_flag)) { ok = false; break; }
+        {
+          uint8_t* xo = xo_smem + h * 256;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int jj = hf * 8 + j;
+            *reinterpret_cast<float4*>(xo + ((jj ^ (h & 15)) << 4)) =
+                make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb->xout_full);
+        if (tid == 0) {
+          mbar_arrive_expect_tx(&bb->x_full[xb], kXBytes);
+          if (!mbar_wait(&bb->xout_full, g & 1, abort_flag)) { ok = false; break; }
+          bulk_copy_to_peer(x_remote + xb * kXBytes, smem_u32(xo_smem), kXBytes, xfull_remote[xb]);
+          bulk_commit_group();
+        }
         if (!mbar_wait_cluster(&bb->x_full[xb], (g >> 1) & 1, abort_flag)) { ok = false; break; }
         {
           const float4* xr = reinterpret_cast<const float4*>(x_smem + xb * kXBytes + h * 256);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float4 o = xr[j ^ (h & 15)];
+          for (int j = 0; j < 8; ++j) {
+            const float4 o = xr[(hf * 8 + j) ^ (h & 15)];
             s[4 * j] += o.x; s[4 * j + 1] += o.y; s[4 * j + 2] += o.z; s[4 * j + 3] += o.w;
           }
         }
-        mbar_arrive_remote(xfree_remote[xb]);
-        // online softmax over this chunk (log2 domain), lazy rescale
+        // mask, scale, chunk max (combined with the other half of the head)
         if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag)) { ok = false; break; }
-        const unsigned long long vmask = bb->kvmask[stage];
-        float cmax = -INFINITY;
+        const uint32_t vm = static_cast<uint32_t>(bb->kvmask[stage][2 * hf]) |
+                            (static_cast<uint32_t>(bb->kvmask[stage][2 * hf + 1]) << 16);
+        float lmax = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          s[j] = ((vmask >> j) & 1ull) ? s[j] * p.scale_log2 : -INFINITY;
-          cmax = fmaxf(cmax, s[j]);
+        for (int j = 0; j < 32; ++j) {
+          s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
+          lmax = fmaxf(lmax, s[j]);
         }
+        bb->red[g & 1][hf][h] = lmax;
+        named_bar_sync(pair_bar, 64);
+        const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]);
         if (cmax > m_run + kRescaleThresh) {
-          const float factor = exp2f(m_run - cmax);  // 0 when m_run = -inf
+          const float factor = ex2_approx(m_run - cmax);  // 0 when m_run = -inf
           if (c > 0) {
-            // O holds PV(0..c-1): wait for PV(c-1), then scale it in place
+            // O holds PV of the earlier chunks: wait for PV(g-1), scale my 128 columns
             if (!mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
-            for (int blk = 0; blk < 8; ++blk) {
+            for (int blk = 0; blk < 4; ++blk) {
               uint32_t v[32];
-              tmem_ld32<32>(t_lane + kOCol + blk * 32, v);
+              const uint32_t col = kOCol + hf * 128 + blk * 32;
+              tmem_ld32<32>(t_lane + col, v);
               tmem_ld_wait();
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * factor);
-              tmem_st32x32(t_lane + kOCol + blk * 32, v);
+              tmem_st32x32(t_lane + col, v);
             }
             tmem_st_wait();
           }
@@ -398,11 +464,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           m_run = cmax;
         }
         float psum = 0.f, esum = 0.f;
-        uint32_t pk[32];
+        uint32_t pk[16];
+        const bool live = m_run != -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float a = m_run == -INFINITY ? 0.f : exp2f(s[2 * j] - m_run);
-          const float bq = m_run == -INFINITY ? 0.f : exp2f(s[2 * j + 1] - m_run);
+        for (int j = 0; j < 16; ++j) {
+          const float a = live ? ex2_approx(s[2 * j] - m_run) : 0.f;
+          const float bq = live ? ex2_approx(s[2 * j + 1] - m_run) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, bq);
           const float2 pf = __bfloat1622float2(pr);
           psum += pf.x + pf.y;
@@ -411,48 +478,71 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         }
         l_run += psum;
         l_lse += esum;
-        // P buffer xb was last read by PV(g-2)
-        if (g >= 2 && !mbar_wait(&bb->pv_done[xb], ((g - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-        {
-          uint8_t* prow = p_smem + xb * kPBytes + h * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(prow + ((j ^ (h & 7)) << 4)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
+        // P lives in TMEM (A operand of PV); PV(g-1) must have finished reading it
+        if (g >= 1 && !mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32x16(t_lane + kPCol + hf * 16, pk);
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bb->p_full[xb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb->p_full[xb]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16
+      // combine the two halves' sums
+      bb->lsum[0][hf][h] = l_run;
+      bb->lsum[1][hf][h] = l_lse;
+      named_bar_sync(pair_bar, 64);
+      const float l_tot = l_run + bb->lsum[0][hf ^ 1][h];
+      const float l_lse_tot = l_lse + bb->lsum[1][hf ^ 1][h];
+      named_bar_sync(pair_bar, 64);  // lsum is rewritten by the next item
+      // epilogue: O / l
       if (!mbar_wait(&bb->o_full, it_n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float lse_v = l_lse_tot > 0.f ? (m_run + __log2f(l_lse_tot)) * 0.6931471805599453f : -INFINITY;
+      if (!partial) {
+        __nv_bfloat16* orow = p.out + (static_cast<size_t>(it.row) * kNH + h) * kDV + rank * 256 + hf * 128;
 #pragma unroll 1
-      for (int blk = 0; blk < 8; ++blk) {
-        uint32_t v[32];
-        tmem_ld32<32>(t_lane + kOCol + blk * 32, v);
-        tmem_ld_wait();
-        uint32_t o[16];
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t v[32];
+          tmem_ld32<32>(t_lane + kOCol + hf * 128 + blk * 32, v);
+          tmem_ld_wait();
+          uint32_t o[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * inv,
-                                                          __uint_as_float(v[2 * j + 1]) * inv);
-          o[j] = *reinterpret_cast<const uint32_t*>(&pr);
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * inv,
+                                                            __uint_as_float(v[2 * j + 1]) * inv);
+            o[j] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + blk * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + blk * 32);
+        if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = lse_v;
+      } else {
+        const size_t slot = static_cast<size_t>(it.row) * p.S + it.split;
+        float* po = p.part_o + (slot * kNH + h) * kDV + rank * 256 + hf * 128;
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t v[32];
+          tmem_ld32<32>(t_lane + kOCol + hf * 128 + blk * 32, v);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(po + blk * 32);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(v[4 * j]) * inv, __uint_as_float(v[4 * j + 1]) * inv,
+                                 __uint_as_float(v[4 * j + 2]) * inv, __uint_as_float(v[4 * j + 3]) * inv);
+        }
+        if (rank == 0 && hf == 0) p.part_lse[slot * kNH + h] = lse_v;
       }
       tc_fence_before();
-      mbar_arrive(&bb->o_free);
-      if (p.lse && rank == 0)
-        p.lse[row * kNH + h] = l_lse > 0.f ? (m_run + log2f(l_lse)) * 0.6931471805599453f : -INFINITY;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bb->o_free);
       ++it_n;
     }
   }
 
+  if (threadIdx.x == 0) bulk_wait_read_all();  // the last partial DMA has read X_out
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, 1u);
@@ -464,44 +554,124 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   }
 }
 
+// Combines the S key-range partials of each row: out = sum_j w_j o_j with
+// w_j = exp(lse_j - LSE), LSE = log sum_j exp(lse_j).
+constexpr int kMergeHeads = 4;
+__global__ void __launch_bounds__(128)
+mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int S) {
+  const size_t row = blockIdx.x;
+  const int h0 = blockIdx.y * kMergeHeads;
+  __shared__ float wgt[kMergeHeads][32];
+  __shared__ float lse_tot[kMergeHeads];
+  if (threadIdx.x < kMergeHeads) {
+    const int h = h0 + threadIdx.x;
+    float m = -INFINITY;
+    for (int j = 0; j < S; ++j) m = fmaxf(m, part_lse[(row * S + j) * kNH + h]);
+    float z = 0.f;
+    for (int j = 0; j < S; ++j) {
+      const float l = part_lse[(row * S + j) * kNH + h];
+      const float e = m == -INFINITY ? 0.f : __expf(l - m);
+      wgt[threadIdx.x][j] = e;
+      z += e;
+    }
+    for (int j = 0; j < S; ++j) wgt[threadIdx.x][j] = z > 0.f ? wgt[threadIdx.x][j] / z : 0.f;
+    lse_tot[threadIdx.x] = z > 0.f ? m + __logf(z) : -INFINITY;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kMergeHeads * kDV / 4; e += blockDim.x) {
+    const int hh = e / (kDV / 4);
+    const int c4 = e % (kDV / 4);
+    const int h = h0 + hh;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < S; ++j) {
+      const float wj = wgt[hh][j];
+      if (wj == 0.f) continue;
+      const float4 v = reinterpret_cast<const float4*>(part_o + ((row * S + j) * kNH + h) * kDV)[c4];
+      acc.x += wj * v.x; acc.y += wj * v.y; acc.z += wj * v.z; acc.w += wj * v.w;
+    }
+    __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y), b2 = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&a);
+    pk.y = *reinterpret_cast<uint32_t*>(&b2);
+    reinterpret_cast<uint2*>(out + (row * kNH + h) * kDV)[c4] = pk;
+  }
+  if (lse && threadIdx.x < kMergeHeads) lse[row * kNH + h0 + threadIdx.x] = lse_tot[threadIdx.x];
+}
+
+struct MlaSplit {
+  int S, cps, pairs;
+};
+
+MlaSplit mla_split(long long rows, int k, int sms) {
+  MlaSplit sp{};
+  const int max_pairs = std::max(1, sms / 2);
+  const int nch = std::max(1, (k + kChunk - 1) / kChunk);
+  sp.S = 1;
+  sp.cps = nch;
+  if (rows < max_pairs) {
+    int S = static_cast<int>(std::min<long long>(32, max_pairs / rows));
+    S = std::max(1, std::min(S, nch));
+    sp.cps = (nch + S - 1) / S;
+    sp.S = (nch + sp.cps - 1) / sp.cps;
+  }
+  sp.pairs = static_cast<int>(std::min<long long>(rows * sp.S, max_pairs));
+  return sp;
+}
+
 }  // namespace
 
-size_t sparse_attn_ws_bytes(int, int, int, int, int) { return 0; }
+size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k) {
+  if (n_h != kNH || D_v != kDV) return 0;
+  const long long rows = static_cast<long long>(B) * Lq;
+  // sized for up to 160 SMs so the requirement does not depend on the device
+  const MlaSplit sp = mla_split(rows, k, 160);
+  if (sp.S <= 1) return 0;
+  return static_cast<size_t>(rows) * sp.S * kNH * (kDV + 1) * sizeof(float) + 256;
+}
 
 dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
                               const dsa_bf16* vbuf, int64_t v_row_stride, const int32_t* idx,
                               int B, int Lq, int Lk, int start_pos, int n_h, int D_qk, int D_v,
                               int k, float scale, dsa_bf16* out, float* lse, void* ws,
                               size_t ws_bytes, cudaStream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   const long long rows = static_cast<long long>(B) * Lq;
   if (rows > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
   const bool mla = n_h == kNH && D_qk == kDQK && D_v == kDV && kbuf == vbuf &&
                    k_row_stride == v_row_stride;
   if (mla) {
-    CUtensorMap tkv;
-    if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(B) * Lk,
-                         static_cast<uint64_t>(k_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
-      return set_error(DSA_ERR_CUDA, "tensor map for the latent cache failed");
+    const int sms = device_sm_count();
+    if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
+    const MlaSplit sp = mla_split(rows, k, std::min(sms, 160));
+    if (rows * sp.S > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
+    const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV + 1) * sizeof(float) : 0;
+    if (need > ws_bytes || (need && !ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_sparse_attn: workspace too small");
     MlaParams p{};
+    p.kv = reinterpret_cast<const __nv_bfloat16*>(kbuf);
+    p.kv_stride = k_row_stride;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.idx = idx;
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.lse = lse;
+    p.part_o = sp.S > 1 ? static_cast<float*>(ws) : nullptr;
+    p.part_lse = sp.S > 1 ? static_cast<float*>(ws) + static_cast<size_t>(rows) * sp.S * kNH * kDV : nullptr;
     p.err = device_error_word();
     if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
     p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k;
+    p.S = sp.S; p.cps = sp.cps;
     p.scale_log2 = scale * 1.4426950408889634f;
-    const int sms = device_sm_count();
-    if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
-    const long long pairs = std::min<long long>(rows, sms / 2);
     cudaError_t e = cudaFuncSetAttribute(mla_sparse_attn_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla smem attribute: ") + cudaGetErrorString(e));
-    mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * pairs), kMlaThreads, kMlaSmem, stream>>>(tkv, p);
+    mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * sp.pairs), kMlaThreads, kMlaSmem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla launch: ") + cudaGetErrorString(e));
+    if (sp.S > 1) {
+      mla_merge_kernel<<<dim3(static_cast<unsigned>(rows), kNH / kMergeHeads), 128, 0, stream>>>(
+          p.part_o, p.part_lse, p.out, lse, sp.S);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla merge launch: ") + cudaGetErrorString(e));
+    }
     return DSA_OK;
   }
   if (n_h <= 128 && D_qk <= 128 && D_v <= 128) {

@@ -186,3 +186,19 @@ def test_mla_full_size_layer_sampled(dsa, oracle_mod):
                           sigma=0.5, corr=True)
         o, _ = oracle_mod.sparse_attn_row(qrow, kv_h[0], kv_h[0], sel[i], scale, Dv=512)
         _close(out[0, i].float().cpu().numpy(), o)
+
+
+def test_mla_split_rows_with_empty_splits(dsa, oracle_mod):
+    # Few rows: the index list is split across clusters and merged; rows that
+    # see only one chunk leave most splits empty.
+    B, Lq, Lk, start_pos, k = 4, 2, 60, 50, 2048
+    rng = np.random.default_rng(15)
+    q, kv = _mla_inputs(16, B, Lq, Lk)
+    idx = _random_rows(rng, B, Lq, start_pos, k)
+    scale = 1 / math.sqrt(576)
+    got, lse = _run_mla(dsa, q, kv, idx, start_pos, scale)
+    for b in range(B):
+        for i in range(Lq):
+            o, l = oracle_mod.sparse_attn_row(q[b, i], kv[b], kv[b], idx[b, i], scale, Dv=512)
+            _close(got[b, i], o)
+            np.testing.assert_allclose(lse[b, i], l, rtol=1e-4, atol=1e-4)

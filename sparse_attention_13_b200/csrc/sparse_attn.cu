@@ -32,6 +32,7 @@
 // simt_sparse_attn_kernel: plain CUDA-core kernel for small head dims
 // (D_qk, D_v <= 128, separate K and V tensors), one block per query row.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cmath>
@@ -107,21 +108,25 @@ constexpr int kSlabBytes = kChunk * 128;       // one 64-column slab of a chunk,
 constexpr int kMaxSlabs = 5;                   // CTA0: columns 0..255, CTA1: 256..575
 constexpr int kStageBytes = kMaxSlabs * kSlabBytes;
 constexpr int kStages = 3;
-constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile fp32
-// TMEM columns: O (fp32, 256) | S (fp32, 64) | P (bf16 pairs, 32) | Q (bf16 pairs, 128 or 160)
-constexpr uint32_t kOCol = 0, kSCol = 256, kPCol = 320, kQCol = 352;
-constexpr int kSoftWarps = 8;
-constexpr int kProdWarp0 = 8, kProdWarps = 4, kMmaWarpA = 12;
-constexpr int kMlaThreads = 416;
+constexpr int kXBytes = kNH * kChunk * 2;      // partial score tile, fp16
+constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, bf16
+// TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64; P(c) overwrites
+// the first 32 columns of S(c) as bf16 pairs) | Q (bf16 pairs, 128)
+constexpr uint32_t kOCol = 0, kSCol = 256, kQCol = 384;
+constexpr int kSoftWarps = 8;                  // warps 0..7
+constexpr int kSendWarp0 = 8, kSendWarps = 4;  // warps 8..11
+constexpr int kProdWarp0 = 12, kProdWarps = 4; // warps 12..15
+constexpr int kMmaWarpA = 16;
+constexpr int kMlaThreads = 17 * 32;
 constexpr float kRescaleThresh = 8.0f;          // log2 units
-constexpr int kPairBarBase = 2;                 // named barriers 2..5: the two warps of a quadrant
+constexpr int kPairBarBase = 2;                 // named barriers 2..5 and 6..9: the two softmax warps of a quadrant
+constexpr int kSendBar = 10;                    // named barriers 10, 11: the sender warps
 
 struct MlaBars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full, s_free;
-  uint64_t p_full[2], pv_done[2];
+  uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
   uint64_t o_full, o_free, q_full;
-  uint64_t x_full[2], xout_full, xout_free;
+  uint64_t x_full[2], x_free[2];
   unsigned short kvmask[kStages][4];            // per producer warp: 16 rows each
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
   float lsum[2][2][kNH];                        // [kind][half][head] final sums
@@ -129,8 +134,8 @@ struct MlaBars {
   int abort_flag;
 };
 
-// shared memory: gather ring | peer partials (double-buffered) | own partial staging
-constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 3 * kXBytes +
+// shared memory: gather ring | peer partials X_in[2] | own partials X_out[2] | Q rope
+constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 4 * kXBytes + kQRopeBytes +
                          static_cast<int>(sizeof(MlaBars)) + 64;
 
 struct MlaParams {
@@ -172,9 +177,10 @@ mla_sparse_attn_kernel(const MlaParams p) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* kv_smem = smem;
-  uint8_t* x_smem = kv_smem + kStages * kStageBytes;   // X_in[2]: the peer's partials
-  uint8_t* xo_smem = x_smem + 2 * kXBytes;             // X_out: this CTA's partial
-  MlaBars* bb = reinterpret_cast<MlaBars*>(xo_smem + kXBytes);
+  uint8_t* xin_smem = kv_smem + kStages * kStageBytes;   // X_in[2]: the peer's partials
+  uint8_t* xout_smem = xin_smem + 2 * kXBytes;           // X_out[2]: this CTA's partials
+  uint8_t* qrope_smem = xout_smem + 2 * kXBytes;         // CTA1: Q[:, 512:576]
+  MlaBars* bb = reinterpret_cast<MlaBars*>(qrope_smem + kQRopeBytes);
   volatile int* abort_flag = &bb->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +192,6 @@ mla_sparse_attn_kernel(const MlaParams p) {
   // CTA0 owns latent columns 0..255 (QK and V), CTA1 owns 256..575 (QK) and
   // 256..511 (V); together they gather each selected row exactly once.
   const int n_slabs = rank == 0 ? 4 : 5;
-  const int qk_steps = n_slabs * 4;
   const int col0 = rank == 0 ? 0 : 256;
 
   if (threadIdx.x == 0) {
@@ -196,18 +201,17 @@ mla_sparse_attn_kernel(const MlaParams p) {
       mbar_init(&bb->kv_full[s], kProdWarps * 32 + kProdWarps);
       mbar_init(&bb->kv_empty[s], 1);
     }
-    mbar_init(&bb->s_full, 1);
-    mbar_init(&bb->s_free, kSoftWarps);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&bb->s_full[b], 1);
+      mbar_init(&bb->s_read[b], kSendWarps);
       mbar_init(&bb->p_full[b], kSoftWarps);
       mbar_init(&bb->pv_done[b], 1);
       mbar_init(&bb->x_full[b], 1);
+      mbar_init(&bb->x_free[b], kSoftWarps);
     }
-    mbar_init(&bb->xout_full, kSoftWarps);
-    mbar_init(&bb->xout_free, 1);
     mbar_init(&bb->o_full, 1);
     mbar_init(&bb->o_free, kSoftWarps);
-    mbar_init(&bb->q_full, kSoftWarps);
+    mbar_init(&bb->q_full, kSendWarps);
     bb->abort_flag = 0;
     fence_barrier_init();
   }
@@ -247,7 +251,8 @@ mla_sparse_attn_kernel(const MlaParams p) {
         const int srow = valid ? sidx : 0;
         const unsigned m = __ballot_sync(0xffffffffu, valid) & 0xffffu;
         if (c + 1 < it.c0 + it.n) s_next = fetch(c + 1);   // overlap the next chunk's index load
-        if (!mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag)) { ok = false; break; }
+        const bool w = __all_sync(0xffffffffu, mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag));
+        if (!w) { ok = false; break; }  // warp-uniform
         const uint32_t dst = smem_u32(kv_smem + stage * kStageBytes);
 #pragma unroll 4
         for (int rr = 0; rr < 16; ++rr) {
@@ -276,20 +281,22 @@ mla_sparse_attn_kernel(const MlaParams p) {
       bool ok = true;
       const uint32_t idesc_qk = make_idesc_bf16(128, kChunk, 0, 0);
       const uint32_t idesc_pv = make_idesc_bf16(128, 256, 0, 1);
+      const uint32_t qrope_base = smem_u32(qrope_smem);
       auto issue_pv = [&](uint32_t gc, bool first) -> bool {
-        const int pb = gc & 1;
-        if (!mbar_wait(&bb->p_full[pb], (gc >> 1) & 1, abort_flag)) return false;
+        const int sb = gc & 1;
+        if (!mbar_wait(&bb->p_full[sb], (gc >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const int stage = gc % kStages;
         // V = this CTA's slabs 0..3: value columns 0..255 (CTA0) or 256..511 (CTA1);
-        // A = P (bf16) in TMEM, 8 columns per 16 rows of the chunk
+        // A = P(gc) (bf16) in the first 32 TMEM columns of S[gc & 1]
         const uint32_t v_base = smem_u32(kv_smem + stage * kStageBytes);
+        const uint32_t p_col = kSCol + sb * 64;
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk) {
           const uint64_t bd = make_smem_desc(v_base + kk * 2048, kSlabBytes, 1024, kSwizzle128B);
-          umma_bf16_ts(tmem + kOCol, tmem + kPCol + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          umma_bf16_ts(tmem + kOCol, tmem + p_col + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
-        umma_commit(&bb->pv_done[pb]);
+        umma_commit(&bb->pv_done[sb]);
         umma_commit(&bb->kv_empty[stage]);
         return true;
       };
@@ -301,15 +308,26 @@ mla_sparse_attn_kernel(const MlaParams p) {
         for (int c = 0; c < it.n && ok; ++c, ++g) {
           const int stage = g % kStages;
           if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&bb->s_free, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          // S[g & 1] was last read by PV(g - 2), issued before this QK (in-order)
           const uint32_t kb = smem_u32(kv_smem + stage * kStageBytes);
-          for (int st = 0; st < qk_steps; ++st) {
+          const uint32_t s_col = kSCol + (g & 1) * 64;
+#pragma unroll
+          for (int st = 0; st < 16; ++st) {
             const uint64_t bd = make_smem_desc(kb + (st >> 2) * kSlabBytes + (st & 3) * 32, 16, 1024,
                                                kSwizzle128B);
-            umma_bf16_ts(tmem + kSCol, tmem + kQCol + st * 8, bd, idesc_qk, st != 0);
+            umma_bf16_ts(tmem + s_col, tmem + kQCol + st * 8, bd, idesc_qk, st != 0);
           }
-          umma_commit(&bb->s_full);
+          if (rank == 1) {
+            // query columns 512..575 from shared memory against slab 4
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = make_smem_desc(qrope_base + kk * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = make_smem_desc(kb + 4 * kSlabBytes + kk * 32, 16, 1024, kSwizzle128B);
+              umma_bf16_ss(tmem + s_col, ad, bd, idesc_qk, 1u);
+            }
+          }
+          umma_commit(&bb->s_full[g & 1]);
           if (c >= 1) {
             if (c == 1 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag)) { ok = false; break; }
             if (!issue_pv(g - 1, c == 1)) { ok = false; break; }
@@ -322,20 +340,118 @@ mla_sparse_attn_kernel(const MlaParams p) {
         ++it_n;
       }
     }
+  } else if (warp >= kSendWarp0) {
+    // ------------------------------------------------------------ sender
+    // thread = head (TMEM lane); loads the CTA's query part at item start and
+    // ships every chunk's partial scores to the peer as soon as QK finishes,
+    // so the exchange overlaps the softmax of the previous chunk.
+    const int qd = warp - kSendWarp0;
+    const int h = qd * 32 + lane;
+    const int stid = threadIdx.x - kSendWarp0 * 32;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const uint32_t xin_remote = mapa_shared(smem_u32(xin_smem), peer);
+    const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bb->x_full[0]), peer),
+                                      mapa_shared(smem_u32(&bb->x_full[1]), peer)};
+    // A failed (timed-out) wait only clears `ok`; the sender warps leave their
+    // loops together, at the next named barrier, so none is left waiting there.
+    uint32_t g = 0, it_n = 0;
+    bool ok = true;
+    for (int item = pair; item < n_items; item += n_pairs) {
+      const MlaItem it = mla_item(p, item);
+      if (it.n == 0) continue;
+      // the previous item's MMAs (which read Q) are complete once its O is
+      if (it_n > 0 && ok) ok = mbar_wait(&bb->o_full, (it_n - 1) & 1, abort_flag);
+      tc_fence_after();
+      if (ok) {
+        const uint4* qsrc = reinterpret_cast<const uint4*>(
+            p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0);
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 v = __ldg(qsrc + blk * 8 + j);
+            r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+          }
+          tmem_st32x32(t_lane + kQCol + blk * 32, r);
+        }
+        if (rank == 1) {
+          // columns 512..575 -> 128B-swizzled K-major row h of the rope tile
+          uint8_t* dst = qrope_smem + h * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(dst + ((j ^ (h & 7)) << 4)) = __ldg(qsrc + 32 + j);
+          fence_proxy_async_smem();
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&bb->q_full);
+      for (int c = 0; c < it.n; ++c, ++g) {
+        const int sb = g & 1;
+        if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
+        tc_fence_after();
+        uint32_t hv[32];
+        if (ok) {
+          uint32_t v[32];
+          tmem_ld32<32>(t_lane + kSCol + sb * 64, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hv[j] = pack_half2_sat(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+          tmem_ld32<32>(t_lane + kSCol + sb * 64 + 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hv[16 + j] = pack_half2_sat(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&bb->s_read[sb]);
+        // X_out[sb] was last read by the DMA of chunk g-2
+        if (stid == 0) bulk_wait_read_allbut1();
+        ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
+        if (!ok) break;
+        {
+          uint8_t* xo = xout_smem + sb * kXBytes + h * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(xo + ((j ^ (h & 7)) << 4)) =
+                make_uint4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(kSendBar + 1, kSendWarps * 32);
+        if (stid == 0) {
+          // the peer consumed its X_in[sb] from chunk g-2; this CTA expects
+          // the peer's partial of chunk g in its own X_in[sb]
+          if (mbar_wait_cluster(&bb->x_free[sb], ((g >> 1) & 1) ^ 1, abort_flag)) {
+            mbar_arrive_expect_tx(&bb->x_full[sb], kXBytes);
+            bulk_copy_to_peer(xin_remote + sb * kXBytes, smem_u32(xout_smem + sb * kXBytes), kXBytes,
+                              xfull_remote[sb]);
+            bulk_commit_group();
+          } else {
+            ok = false;  // the abort flag is raised; the next barrier ends the loop
+          }
+        }
+      }
+      ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
+      if (!ok) break;
+      ++it_n;
+    }
+    if (stid == 0) bulk_wait_read_all();  // the last DMA has read X_out
   } else {
     // ------------------------------------------------------------ softmax
     // thread = (head h = TMEM lane, half hf of the chunk's 64 columns)
     const int qd = warp & 3, hf = warp >> 2;
     const int h = qd * 32 + lane;
-    const int tid = threadIdx.x;
     const int pair_bar = kPairBarBase + qd;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const uint32_t x_remote = mapa_shared(smem_u32(x_smem), peer);
-    const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bb->x_full[0]), peer),
-                                      mapa_shared(smem_u32(&bb->x_full[1]), peer)};
+    const uint32_t xfree_remote[2] = {mapa_shared(smem_u32(&bb->x_free[0]), peer),
+                                      mapa_shared(smem_u32(&bb->x_free[1]), peer)};
+    // A failed (timed-out) wait only clears `ok`; the two warps of a head pair
+    // leave their loops together at the next pair barrier.
     uint32_t g = 0, it_n = 0;
     bool ok = true;
-    for (int item = pair; item < n_items && ok; item += n_pairs) {
+    for (int item = pair; item < n_items; item += n_pairs) {
       const MlaItem it = mla_item(p, item);
       const bool partial = p.S > 1;
       if (it.n == 0) {
@@ -352,112 +468,76 @@ mla_sparse_attn_kernel(const MlaParams p) {
         }
         continue;
       }
-      // this CTA's part of the query row -> TMEM (A operand of QK)
-      {
-        const uint4* qsrc = reinterpret_cast<const uint4*>(
-            p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0 + hf * 128);
-        const int nblk = hf == 0 ? 2 : (rank == 0 ? 2 : 3);
-        for (int blk = 0; blk < nblk; ++blk) {
-          uint32_t r[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 v = __ldg(qsrc + blk * 8 + j);
-            r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
-          }
-          tmem_st32x32(t_lane + kQCol + hf * 64 + blk * 32, r);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bb->q_full);
-      }
       // l_run: sum of the bf16 weights PV multiplies (normalises O);
       // l_lse: the same sum before rounding (for the log-sum-exp).  Each half
       // of a head keeps the sums of its own columns.
       float m_run = -INFINITY, l_run = 0.f, l_lse = 0.f;
       for (int c = 0; c < it.n; ++c, ++g) {
         const int stage = g % kStages;
-        const int xb = g & 1;
-        if (!mbar_wait(&bb->s_full, g & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
+        const int sb = g & 1;
         float s[32];
-        {
+        if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
+        tc_fence_after();
+        if (ok) {
           uint32_t v[32];
-          tmem_ld32<32>(t_lane + kSCol + hf * 32, v);
+          tmem_ld32<32>(t_lane + kSCol + sb * 64 + hf * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bb->s_free);
-        // Partial scores -> peer: stage them in X_out, one thread moves the
-        // whole 32 KB tile with a bulk DMA that completes on the peer's
-        // x_full[xb].  X_in is double-buffered; the peer can only send chunk
-        // g+2 after it received this CTA's chunk g+1, which is sent after
-        // X_in[xb] was consumed below, so no release handshake is needed.
-        if (tid == 0 && g > 0) {
-          bulk_wait_read_all();           // the previous DMA finished reading X_out
-          mbar_arrive(&bb->xout_free);
-        }
-        if (g > 0 && !mbar_wait(&bb->xout_free, (g - 1) & 1, abort_flag)) { ok = false; break; }
-        {
-          uint8_t* xo = xo_smem + h * 256;
+        // + the peer's partial scores of the same columns (fp16)
+        if (ok) ok = mbar_wait_cluster(&bb->x_full[sb], (g >> 1) & 1, abort_flag);
+        if (ok) {
+          const uint8_t* xr = xin_smem + sb * kXBytes + h * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int jj = hf * 8 + j;
-            *reinterpret_cast<float4*>(xo + ((jj ^ (h & 15)) << 4)) =
-                make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+          for (int j = 0; j < 4; ++j) {
+            const uint4 o = *reinterpret_cast<const uint4*>(xr + (((hf * 4 + j) ^ (h & 7)) << 4));
+            const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
+              s[8 * j + 2 * e] += f.x;
+              s[8 * j + 2 * e + 1] += f.y;
+            }
           }
         }
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bb->xout_full);
-        if (tid == 0) {
-          mbar_arrive_expect_tx(&bb->x_full[xb], kXBytes);
-          if (!mbar_wait(&bb->xout_full, g & 1, abort_flag)) { ok = false; break; }
-          bulk_copy_to_peer(x_remote + xb * kXBytes, smem_u32(xo_smem), kXBytes, xfull_remote[xb]);
-          bulk_commit_group();
-        }
-        if (!mbar_wait_cluster(&bb->x_full[xb], (g >> 1) & 1, abort_flag)) { ok = false; break; }
-        {
-          const float4* xr = reinterpret_cast<const float4*>(x_smem + xb * kXBytes + h * 256);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 o = xr[(hf * 8 + j) ^ (h & 15)];
-            s[4 * j] += o.x; s[4 * j + 1] += o.y; s[4 * j + 2] += o.z; s[4 * j + 3] += o.w;
-          }
-        }
+        if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote[sb]);
         // mask, scale, chunk max (combined with the other half of the head)
-        if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t vm = static_cast<uint32_t>(bb->kvmask[stage][2 * hf]) |
-                            (static_cast<uint32_t>(bb->kvmask[stage][2 * hf + 1]) << 16);
+        if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
         float lmax = -INFINITY;
+        if (ok) {
+          const uint32_t vm = static_cast<uint32_t>(bb->kvmask[stage][2 * hf]) |
+                              (static_cast<uint32_t>(bb->kvmask[stage][2 * hf + 1]) << 16);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
-          lmax = fmaxf(lmax, s[j]);
+          for (int j = 0; j < 32; ++j) {
+            s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
+            lmax = fmaxf(lmax, s[j]);
+          }
         }
         bb->red[g & 1][hf][h] = lmax;
-        named_bar_sync(pair_bar, 64);
+        ok = named_bar_and(pair_bar, 64, ok);
+        if (!ok) break;
         const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]);
         if (cmax > m_run + kRescaleThresh) {
           const float factor = ex2_approx(m_run - cmax);  // 0 when m_run = -inf
           if (c > 0) {
             // O holds PV of the earlier chunks: wait for PV(g-1), scale my 128 columns
-            if (!mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+            ok = mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag);
             tc_fence_after();
+            if (ok) {
 #pragma unroll 1
-            for (int blk = 0; blk < 4; ++blk) {
-              uint32_t v[32];
-              const uint32_t col = kOCol + hf * 128 + blk * 32;
-              tmem_ld32<32>(t_lane + col, v);
-              tmem_ld_wait();
+              for (int blk = 0; blk < 4; ++blk) {
+                uint32_t v[32];
+                const uint32_t col = kOCol + hf * 128 + blk * 32;
+                tmem_ld32<32>(t_lane + col, v);
+                tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * factor);
-              tmem_st32x32(t_lane + col, v);
+                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * factor);
+                tmem_st32x32(t_lane + col, v);
+              }
+              tmem_st_wait();
             }
-            tmem_st_wait();
           }
           l_run *= factor;
           l_lse *= factor;
@@ -478,29 +558,32 @@ mla_sparse_attn_kernel(const MlaParams p) {
         }
         l_run += psum;
         l_lse += esum;
-        // P lives in TMEM (A operand of PV); PV(g-1) must have finished reading it
-        if (g >= 1 && !mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        // P(g) overwrites the first 32 columns of S[g & 1] once the sender has
+        // read them (both halves of this head read theirs before the pair barrier)
+        if (ok) ok = mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag);
         tc_fence_after();
-        tmem_st32x16(t_lane + kPCol + hf * 16, pk);
-        tmem_st_wait();
+        if (ok) {
+          tmem_st32x16(t_lane + kSCol + sb * 64 + hf * 16, pk);
+          tmem_st_wait();
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bb->p_full[xb]);
+        if (lane == 0 && ok) mbar_arrive(&bb->p_full[sb]);
       }
-      if (!ok) break;
       // combine the two halves' sums
       bb->lsum[0][hf][h] = l_run;
       bb->lsum[1][hf][h] = l_lse;
-      named_bar_sync(pair_bar, 64);
+      ok = named_bar_and(pair_bar, 64, ok);
+      if (!ok) break;
       const float l_tot = l_run + bb->lsum[0][hf ^ 1][h];
       const float l_lse_tot = l_lse + bb->lsum[1][hf ^ 1][h];
-      named_bar_sync(pair_bar, 64);  // lsum is rewritten by the next item
+      named_bar_sync(pair_bar + 4, 64);  // lsum is rewritten by the next item
       // epilogue: O / l
-      if (!mbar_wait(&bb->o_full, it_n & 1, abort_flag)) { ok = false; break; }
+      ok = mbar_wait(&bb->o_full, it_n & 1, abort_flag);
       tc_fence_after();
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float lse_v = l_lse_tot > 0.f ? (m_run + __log2f(l_lse_tot)) * 0.6931471805599453f : -INFINITY;
-      if (!partial) {
+      if (ok && !partial) {
         __nv_bfloat16* orow = p.out + (static_cast<size_t>(it.row) * kNH + h) * kDV + rank * 256 + hf * 128;
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
@@ -519,7 +602,7 @@ mla_sparse_attn_kernel(const MlaParams p) {
           for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         }
         if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = lse_v;
-      } else {
+      } else if (ok) {
         const size_t slot = static_cast<size_t>(it.row) * p.S + it.split;
         float* po = p.part_o + (slot * kNH + h) * kDV + rank * 256 + hf * 128;
 #pragma unroll 1
@@ -537,12 +620,11 @@ mla_sparse_attn_kernel(const MlaParams p) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bb->o_free);
+      if (lane == 0 && ok) mbar_arrive(&bb->o_free);
       ++it_n;
     }
   }
 
-  if (threadIdx.x == 0) bulk_wait_read_all();  // the last partial DMA has read X_out
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, 1u);

@@ -14,6 +14,11 @@ from gpu_util import to_dev_bf16
 pytestmark = pytest.mark.gpu
 
 ATOL, RTOL = 2e-2, 1e-2
+# MLA log-sum-exp: each CTA of a pair adds the peer's half of every score as
+# fp16 (relative rounding <= 2^-11), so a logit moves by at most
+# scale * 2^-11 * |partial score|; with 576-wide N(0, 0.5^2) rows the partial
+# scores stay below ~40, giving |dLSE| <= 1/24 * 2^-11 * 40 ~ 1e-3.
+LSE_ATOL = 1e-3
 
 
 @pytest.fixture(scope="module")
@@ -111,7 +116,7 @@ def test_mla_short_rows_equal_dense(dsa, oracle_mod):
         for i in list(range(1, 12)) + [63, 64, 65, 100, 127, 128, 129, 149]:
             o, l = oracle_mod.dense_attn_row(q[b, i], kv[b], kv[b], i, scale, Dv=512)
             _close(got[b, i], o)
-            np.testing.assert_allclose(lse[b, i], l, rtol=1e-4, atol=1e-4)
+            np.testing.assert_allclose(lse[b, i], l, rtol=0, atol=LSE_ATOL)
 
 
 @pytest.mark.parametrize("holes", [False, True])
@@ -126,7 +131,7 @@ def test_mla_random_subsets(dsa, oracle_mod, holes):
         o, l = oracle_mod.sparse_attn_row(q[0, i], kv[0], kv[0], idx[0, i], scale, Dv=512)
         _close(got[0, i], o)
         if i > 0:
-            np.testing.assert_allclose(lse[0, i], l, rtol=1e-4, atol=1e-4)
+            np.testing.assert_allclose(lse[0, i], l, rtol=0, atol=LSE_ATOL)
 
 
 def test_mla_decode_rows(dsa, oracle_mod):
@@ -139,7 +144,7 @@ def test_mla_decode_rows(dsa, oracle_mod):
     for b in range(B):
         o, l = oracle_mod.sparse_attn_row(q[b, 0], kv[b], kv[b], idx[b, 0], scale, Dv=512)
         _close(got[b, 0], o)
-        np.testing.assert_allclose(lse[b, 0], l, rtol=1e-4, atol=1e-4)
+        np.testing.assert_allclose(lse[b, 0], l, rtol=0, atol=LSE_ATOL)
 
 
 def test_mla_deterministic(dsa):
@@ -201,4 +206,4 @@ def test_mla_split_rows_with_empty_splits(dsa, oracle_mod):
         for i in range(Lq):
             o, l = oracle_mod.sparse_attn_row(q[b, i], kv[b], kv[b], idx[b, i], scale, Dv=512)
             _close(got[b, i], o)
-            np.testing.assert_allclose(lse[b, i], l, rtol=1e-4, atol=1e-4)
+            np.testing.assert_allclose(lse[b, i], l, rtol=0, atol=LSE_ATOL)

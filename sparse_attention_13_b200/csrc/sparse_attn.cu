@@ -10,8 +10,8 @@
 //   at a time.  CTA0 holds latent columns 0..255 of the query in TMEM, CTA1
 //   columns 256..575 (the A operand of the QK UMMA); CTA c accumulates output
 //   columns 256c..256c+255 in TMEM (fp32).  Per chunk of 64 selected rows:
-//     4 producer warps  cp.async gather of the chunk's latent rows (CTA0: 4
-//                    slabs of 64 columns, CTA1: 5 slabs) into the 128B-swizzled
+//     8 producer warps  TMA gather4 of the chunk's latent rows (CTA0: 4 slabs
+//                    of 64 columns, CTA1: 5 slabs) into the 128B-swizzled
 //                    layout, 3-stage ring; each selected row is read from
 //                    memory exactly once;
 //     MMA warp       S_c = Q_c K_c^T over the CTA's columns (A from TMEM),
@@ -115,9 +115,9 @@ constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, 
 constexpr uint32_t kOCol = 0, kSCol = 256, kQCol = 384;
 constexpr int kSoftWarps = 8;                  // warps 0..7
 constexpr int kSendWarp0 = 8, kSendWarps = 4;  // warps 8..11
-constexpr int kProdWarp0 = 12, kProdWarps = 4; // warps 12..15
-constexpr int kMmaWarpA = 16;
-constexpr int kMlaThreads = 17 * 32;
+constexpr int kProdWarp0 = 12, kProdWarps = 7; // warps 12..18: the chunk's 16 four-row groups
+constexpr int kMmaWarpA = 19;
+constexpr int kMlaThreads = 20 * 32;           // 20 warps: 96 registers per thread
 constexpr float kRescaleThresh = 8.0f;          // log2 units
 constexpr int kPairBarBase = 2;                 // named barriers 2..5 and 6..9: the two softmax warps of a quadrant
 constexpr int kSendBar = 10;                    // named barriers 10, 11: the sender warps
@@ -127,7 +127,7 @@ struct MlaBars {
   uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
   uint64_t o_full, o_free, q_full;
   uint64_t x_full[2], x_free[2];
-  unsigned short kvmask[kStages][4];            // per producer warp: 16 rows each
+  unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
   float lsum[2][2][kNH];                        // [kind][half][head] final sums
   uint32_t tmem_slot;
@@ -139,8 +139,6 @@ constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 4 * kXBytes + kQRopeByte
                          static_cast<int>(sizeof(MlaBars)) + 64;
 
 struct MlaParams {
-  const __nv_bfloat16* kv;  // latent rows, row stride kv_stride
-  int64_t kv_stride;
   const __nv_bfloat16* q;   // [B*Lq][128][576]
   const int32_t* idx;       // [B*Lq][k]
   __nv_bfloat16* out;       // [B*Lq][128][512]
@@ -172,7 +170,7 @@ __device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int item) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
-mla_sparse_attn_kernel(const MlaParams p) {
+mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -195,10 +193,9 @@ mla_sparse_attn_kernel(const MlaParams p) {
   const int col0 = rank == 0 ? 0 : 256;
 
   if (threadIdx.x == 0) {
-    // kv_full: one cp.async-completion arrival per producer thread plus one
-    // ordinary arrival per producer warp (after its validity mask is written)
+    // kv_full: one arrive.expect_tx per 4-row group issuer
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bb->kv_full[s], kProdWarps * 32 + kProdWarps);
+      mbar_init(&bb->kv_full[s], kChunk / 4);
       mbar_init(&bb->kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -226,21 +223,24 @@ mla_sparse_attn_kernel(const MlaParams p) {
 
   if (warp >= kProdWarp0 && warp < kProdWarp0 + kProdWarps) {
     // ------------------------------------------------------------ gather
-    // Producer warp pw copies rows 16pw..16pw+15 of each 64-row chunk: per
-    // row, consecutive lanes move consecutive 16-byte pieces of the CTA's
-    // columns into the 128B-swizzled slab layout the UMMAs read.
+    // TMA gather4 of the chunk's selected latent rows into the 128B-swizzled
+    // slab layout the UMMAs read.  Gather throughput grows with the number of
+    // issuing warps, so 7 warps share each chunk's 16 four-row groups: warp pw
+    // owns groups pw, pw + 7 and pw + 14 (when < 16); lane i issues group
+    // pw + 7i over all slabs after lanes 4i..4i+3 fetched its row indices.
     const int pw = warp - kProdWarp0;
-    const int n_pieces = n_slabs * 8;
+    const int n_groups = pw + 14 < 16 ? 3 : 2;
     uint32_t g = 0;  // global chunk counter
     bool ok = true;
     for (int item = pair; item < n_items && ok; item += n_pairs) {
       const MlaItem it = mla_item(p, item);
       if (it.n == 0) continue;
       const int32_t* irow = p.idx + static_cast<size_t>(it.row) * p.k;
-      const __nv_bfloat16* kvb = p.kv + static_cast<int64_t>(it.b) * p.Lk * p.kv_stride + col0;
+      const int row_base = it.b * p.Lk;
+      const int my_group = pw + 7 * (lane >> 2);            // group whose row this lane fetches
       auto fetch = [&](int c) -> int {
-        const int r = c * kChunk + pw * 16 + (lane & 15);
-        return (lane < 16 && r < it.nv) ? __ldg(irow + r) : -1;
+        const int r = c * kChunk + my_group * 4 + (lane & 3);
+        return ((lane >> 2) < n_groups && r < it.nv) ? __ldg(irow + r) : -1;
       };
       int s_next = fetch(it.c0);
       for (int c = it.c0; c < it.c0 + it.n; ++c, ++g) {
@@ -248,31 +248,25 @@ mla_sparse_attn_kernel(const MlaParams p) {
         const uint32_t ph = (g / kStages) & 1;
         const int sidx = s_next;
         const bool valid = sidx >= 0 && sidx < p.Lk;
-        const int srow = valid ? sidx : 0;
-        const unsigned m = __ballot_sync(0xffffffffu, valid) & 0xffffu;
+        const int grow = row_base + (valid ? sidx : 0);   // padded rows read row 0 (masked later)
+        const unsigned m = __ballot_sync(0xffffffffu, valid);
+        const int src = (lane < n_groups ? lane : 0) * 4;
+        const int r0 = __shfl_sync(0xffffffffu, grow, src + 0);
+        const int r1 = __shfl_sync(0xffffffffu, grow, src + 1);
+        const int r2 = __shfl_sync(0xffffffffu, grow, src + 2);
+        const int r3 = __shfl_sync(0xffffffffu, grow, src + 3);
         if (c + 1 < it.c0 + it.n) s_next = fetch(c + 1);   // overlap the next chunk's index load
         const bool w = __all_sync(0xffffffffu, mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag));
         if (!w) { ok = false; break; }  // warp-uniform
-        const uint32_t dst = smem_u32(kv_smem + stage * kStageBytes);
-#pragma unroll 4
-        for (int rr = 0; rr < 16; ++rr) {
-          const int row_s = __shfl_sync(0xffffffffu, srow, rr);
-          const int r = pw * 16 + rr;
-          const __nv_bfloat16* src = kvb + static_cast<int64_t>(row_s) * p.kv_stride;
-          for (int piece = lane; piece < n_pieces; piece += 32) {
-            const int sl = piece >> 3, j = piece & 7;
-            cp_async_16(dst + sl * kSlabBytes + r * 128 + ((j ^ (r & 7)) << 4), src + piece * 8);
-          }
+        if (lane < n_groups) {
+          const int grp = pw + 7 * lane;
+          bb->kvmask[stage][grp] = static_cast<unsigned char>((m >> (4 * lane)) & 0xFu);
+          uint8_t* dst = kv_smem + stage * kStageBytes + grp * 512;
+          mbar_arrive_expect_tx(&bb->kv_full[stage], n_slabs * 512);
+          for (int sl = 0; sl < n_slabs; ++sl)
+            tma_gather4(dst + sl * kSlabBytes, &tm_kv, &bb->kv_full[stage], col0 + sl * 64, r0, r1, r2, r3);
         }
-        if (lane == 0) bb->kvmask[stage][pw] = static_cast<unsigned short>(m);
-        cp_async_arrive_noinc(&bb->kv_full[stage]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bb->kv_full[stage]);
       }
-    }
-    if (!ok) {
-      // abort path: let this thread's copies land before the CTA can exit
-      asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else if (warp == kMmaWarpA) {
     // ------------------------------------------------------------ MMA
@@ -507,8 +501,9 @@ mla_sparse_attn_kernel(const MlaParams p) {
         if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
         float lmax = -INFINITY;
         if (ok) {
-          const uint32_t vm = static_cast<uint32_t>(bb->kvmask[stage][2 * hf]) |
-                              (static_cast<uint32_t>(bb->kvmask[stage][2 * hf + 1]) << 16);
+          uint32_t vm = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vm |= static_cast<uint32_t>(bb->kvmask[stage][8 * hf + i] & 0xFu) << (4 * i);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
@@ -728,9 +723,11 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     if (rows * sp.S > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
     const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV + 1) * sizeof(float) : 0;
     if (need > ws_bytes || (need && !ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_sparse_attn: workspace too small");
+    CUtensorMap tkv;
+    if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(B) * Lk,
+                         static_cast<uint64_t>(k_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+      return set_error(DSA_ERR_CUDA, "tensor map for the latent cache failed");
     MlaParams p{};
-    p.kv = reinterpret_cast<const __nv_bfloat16*>(kbuf);
-    p.kv_stride = k_row_stride;
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.idx = idx;
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -745,7 +742,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     cudaError_t e = cudaFuncSetAttribute(mla_sparse_attn_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla smem attribute: ") + cudaGetErrorString(e));
-    mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * sp.pairs), kMlaThreads, kMlaSmem, stream>>>(p);
+    mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * sp.pairs), kMlaThreads, kMlaSmem, stream>>>(tkv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla launch: ") + cudaGetErrorString(e));
     if (sp.S > 1) {

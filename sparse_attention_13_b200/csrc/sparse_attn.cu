@@ -129,7 +129,7 @@ struct MlaBars {
   uint64_t x_full[2], x_free[2];
   unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
-  float lsum[2][2][kNH];                        // [kind][half][head] final sums
+  float lsum[1][2][kNH];                        // [half][head] final sums
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -462,10 +462,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         }
         continue;
       }
-      // l_run: sum of the bf16 weights PV multiplies (normalises O);
-      // l_lse: the same sum before rounding (for the log-sum-exp).  Each half
-      // of a head keeps the sums of its own columns.
-      float m_run = -INFINITY, l_run = 0.f, l_lse = 0.f;
+      // l_run: softmax denominator (fp32, before the bf16 rounding of P); each
+      // half of a head keeps the sum of its own columns.
+      float m_run = -INFINITY, l_run = 0.f;
       for (int c = 0; c < it.n; ++c, ++g) {
         const int stage = g % kStages;
         const int sb = g & 1;
@@ -495,15 +494,16 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             }
           }
         }
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote[sb]);
         // mask, scale, chunk max (combined with the other half of the head)
         if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
         float lmax = -INFINITY;
         if (ok) {
-          uint32_t vm = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) vm |= static_cast<uint32_t>(bb->kvmask[stage][8 * hf + i] & 0xFu) << (4 * i);
+          // eight 4-bit group masks (one per byte) -> 32 row bits
+          uint64_t x = *reinterpret_cast<const uint64_t*>(&bb->kvmask[stage][8 * hf]) & 0x0F0F0F0F0F0F0F0Full;
+          x = (x | (x >> 4)) & 0x00FF00FF00FF00FFull;
+          x = (x | (x >> 8)) & 0x0000FFFF0000FFFFull;
+          x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
+          const uint32_t vm = static_cast<uint32_t>(x);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
@@ -535,10 +535,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             }
           }
           l_run *= factor;
-          l_lse *= factor;
           m_run = cmax;
         }
-        float psum = 0.f, esum = 0.f;
+        float esum = 0.f;
         uint32_t pk[16];
         const bool live = m_run != -INFINITY;
 #pragma unroll
@@ -546,13 +545,10 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           const float a = live ? ex2_approx(s[2 * j] - m_run) : 0.f;
           const float bq = live ? ex2_approx(s[2 * j + 1] - m_run) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, bq);
-          const float2 pf = __bfloat1622float2(pr);
-          psum += pf.x + pf.y;
           esum += a + bq;
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        l_run += psum;
-        l_lse += esum;
+        l_run += esum;
         // P(g) overwrites the first 32 columns of S[g & 1] once the sender has
         // read them (both halves of this head read theirs before the pair barrier)
         if (ok) ok = mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag);
@@ -563,15 +559,18 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&bb->p_full[sb]);
+        if (lane == 0 && ok) {
+          mbar_arrive(&bb->p_full[sb]);
+          // X_in[sb] was consumed above: the peer may send chunk g+2 into it
+          mbar_arrive_remote_relaxed(xfree_remote[sb]);
+        }
       }
       // combine the two halves' sums
       bb->lsum[0][hf][h] = l_run;
-      bb->lsum[1][hf][h] = l_lse;
       ok = named_bar_and(pair_bar, 64, ok);
       if (!ok) break;
       const float l_tot = l_run + bb->lsum[0][hf ^ 1][h];
-      const float l_lse_tot = l_lse + bb->lsum[1][hf ^ 1][h];
+      const float l_lse_tot = l_tot;
       named_bar_sync(pair_bar + 4, 64);  // lsum is rewritten by the next item
       // epilogue: O / l
       ok = mbar_wait(&bb->o_full, it_n & 1, abort_flag);

@@ -9,6 +9,8 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "dsa_internal.h"
 #include "dsa_ptx.cuh"
@@ -86,6 +88,20 @@ unsigned int* device_error_word() {
     cache[dev] = static_cast<unsigned int*>(p);
   }
   return cache[dev];
+}
+
+cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<int, const void*>, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& d : done)
+    if (d.first.first == dev && d.first.second == func && d.second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({{dev, func}, bytes});
+  return e;
 }
 
 int device_sm_count() {

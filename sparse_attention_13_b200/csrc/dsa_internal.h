@@ -24,6 +24,11 @@ bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
                      uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
                      CUtensorMapSwizzle swizzle);
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, calling the runtime only the first time per (device, kernel)
+// and size (launch paths stay cheap when called every layer).
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+
 // SM count of the current device (cached per device).
 int device_sm_count();
 

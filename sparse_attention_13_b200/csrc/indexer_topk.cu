@@ -133,50 +133,96 @@ __device__ __forceinline__ unsigned long long pack_entry(float score, int s) {
 }
 
 // ------------------------------------------------------------------ select
-// Exact top-k of buf[0, cnt) (distinct uint64 entries in ascending-s order)
-// by all 256 epilogue threads.  mode 0: keep the best k in place (stable),
-// return the k-th largest value.  mode 1: write the selected positions to
-// out_idx (ascending) and pad with -1 up to k.  mode 2: copy the selected
-// entries to out_list and their number to *out_count.
+// Exclusive prefix of per-(row, warp) counts over the 256 epilogue threads in
+// (row, warp, lane) order; writes sh.woff and returns the total.
+__device__ __forceinline__ int scan_rows(const unsigned (&mask)[kSelRows], SelShared& sh) {
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int r = 0; r < kSelRows; ++r)
+    if (lane == 0) sh.wcnt[r][warp] = __popc(mask[r]);
+  named_bar_sync(kEpiBar, kEpiThreads);
+  if (warp == 0) {
+    constexpr int kN = kSelRows * kEpiWarps;
+    constexpr int kPer = (kN + 31) / 32;
+    int loc[kPer];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      loc[i] = e < kN ? (&sh.wcnt[0][0])[e] : 0;
+      sum += loc[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      if (e < kN) (&sh.woff[0][0])[e] = run;
+      run += loc[i];
+    }
+    if (lane == 31) sh.total = incl;
+  }
+  named_bar_sync(kEpiBar, kEpiThreads);
+  return sh.total;
+}
+
+// Exact top-k of buf[0, cnt): distinct uint64 entries (score key << 32 | ~s)
+// held in ascending-position order, by all 256 epilogue threads.  The radix
+// select runs on the 32-bit score key only; entries tied with the threshold
+// key are taken in buffer order, i.e. lowest position first, which is the
+// (score desc, position asc) order.  mode 0: keep the best k in place
+// (stable) and return the smallest kept entry.  mode 1: write the selected
+// positions to out_idx (ascending) and pad with -1 up to k.  mode 2: copy the
+// selected entries to out_list and their number to *out_count.
 __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inplace,
                                           int cnt, int k, int mode, int32_t* out_idx,
                                           uint64_t* out_list, int* out_count, SelShared& sh) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const unsigned lt = (1u << lane) - 1u;
   unsigned long long v[kSelRows];
 #pragma unroll
   for (int r = 0; r < kSelRows; ++r) {
     const int e = r * kEpiThreads + tid;
     v[r] = e < cnt ? src[e] : 0ull;
   }
-  unsigned long long thr = 0ull;  // keep entries >= thr
+  uint32_t thr = 0u;       // threshold score key
+  int ties = 1 << 30;      // how many entries equal to thr are kept (in order)
   if (cnt > k) {
-    unsigned long long prefix = 0ull;
+    uint32_t prefix = 0u;
     int kk = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    bool exact = true;     // the loop ran down to a single key value
+    for (int shift = 24; shift >= 0; shift -= 8) {
       sh.hist[tid] = 0;
       named_bar_sync(kEpiBar, kEpiThreads);
 #pragma unroll
       for (int r = 0; r < kSelRows; ++r) {
         const int e = r * kEpiThreads + tid;
         if (e < cnt) {
-          const bool match = shift == 56 || ((v[r] >> (shift + 8)) == (prefix >> (shift + 8)));
-          if (match) atomicAdd(&sh.hist[(v[r] >> shift) & 255ull], 1);
+          const uint32_t key = static_cast<uint32_t>(v[r] >> 32);
+          if (shift == 24 || (key >> (shift + 8)) == (prefix >> (shift + 8)))
+            atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
         }
       }
       named_bar_sync(kEpiBar, kEpiThreads);
       if (warp == 0) {
         int loc[8];
-        int s = 0;
+        int sum = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { loc[i] = sh.hist[lane * 8 + i]; s += loc[i]; }
-        int incl = s;  // inclusive suffix sum over lanes >= lane
+        for (int i = 0; i < 8; ++i) { loc[i] = sh.hist[lane * 8 + i]; sum += loc[i]; }
+        int incl = sum;  // inclusive suffix sum over lanes >= lane
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const int y = __shfl_down_sync(0xffffffffu, incl, off);
           if (lane + off < 32) incl += y;
         }
-        int above = incl - s;  // entries in bins of higher lanes
+        int above = incl - sum;  // entries in bins of higher lanes
 #pragma unroll
         for (int i = 7; i >= 0; --i) {
           if (above < kk && above + loc[i] >= kk) {
@@ -188,57 +234,43 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
         }
       }
       named_bar_sync(kEpiBar, kEpiThreads);
-      const int bin = sh.sel_bin;
-      prefix |= static_cast<unsigned long long>(bin) << shift;
+      prefix |= static_cast<uint32_t>(sh.sel_bin) << shift;
       kk = sh.kk_new;
-      if (sh.bin_count == kk) break;
+      if (sh.bin_count == kk) {  // the whole bin is selected: keep every key >= prefix
+        exact = false;
+        break;
+      }
     }
     thr = prefix;
+    if (exact) ties = kk;
   }
-  // stable compaction of entries >= thr, row-major over (r, warp, lane)
+  // keep decision: key > thr, or key == thr within the first `ties` such entries
+  bool keep[kSelRows];
   unsigned mask[kSelRows];
+  bool limited = ties < (1 << 30);
 #pragma unroll
   for (int r = 0; r < kSelRows; ++r) {
     const int e = r * kEpiThreads + tid;
-    const bool keep = e < cnt && v[r] >= thr;
-    mask[r] = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) sh.wcnt[r][warp] = __popc(mask[r]);
+    const uint32_t key = static_cast<uint32_t>(v[r] >> 32);
+    keep[r] = e < cnt && (limited ? key > thr : key >= thr);
+    mask[r] = __ballot_sync(0xffffffffu, e < cnt && limited && key == thr);
   }
+  if (limited) {
+    scan_rows(mask, sh);
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r)
+      if (mask[r] & (1u << lane))
+        keep[r] = keep[r] || (sh.woff[r][warp] + __popc(mask[r] & lt) < ties);
+    named_bar_sync(kEpiBar, kEpiThreads);  // woff is reused below
+  }
+#pragma unroll
+  for (int r = 0; r < kSelRows; ++r) mask[r] = __ballot_sync(0xffffffffu, keep[r]);
   if (tid == 0) sh.minval = ~0ull;
-  named_bar_sync(kEpiBar, kEpiThreads);
-  if (warp == 0) {
-    constexpr int kN = kSelRows * kEpiWarps;
-    constexpr int kPer = (kN + 31) / 32;
-    int loc[kPer];
-    int s = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane * kPer + i;
-      loc[i] = e < kN ? (&sh.wcnt[0][0])[e] : 0;
-      s += loc[i];
-    }
-    int incl = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    int run = incl - s;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane * kPer + i;
-      if (e < kN) (&sh.woff[0][0])[e] = run;
-      run += loc[i];
-    }
-    if (lane == 31) sh.total = incl;
-  }
-  named_bar_sync(kEpiBar, kEpiThreads);
-  const int total = sh.total;
-  const unsigned lt = (1u << lane) - 1u;
+  const int total = scan_rows(mask, sh);
   unsigned long long local_min = ~0ull;
 #pragma unroll
   for (int r = 0; r < kSelRows; ++r) {
-    if (mask[r] & (1u << lane)) {
+    if (keep[r]) {
       const int pos = sh.woff[r][warp] + __popc(mask[r] & lt);
       if (mode == 0) {
         dst_inplace[pos] = v[r];
@@ -583,18 +615,49 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ------------------------------------------------------------------ merge
-// Final top-k over the S per-split candidate lists of one query row.
-// Concatenating the lists in split order keeps ascending positions, so a
-// stable filter yields the ascending output row directly.
-constexpr int kMergeThreads = 512;
+// Final top-k over the S per-split candidate lists of one query row.  The
+// lists concatenated in split order are in ascending position order, so the
+// 32-bit score keys are radix-selected in shared memory and ties at the
+// threshold are taken in that order; a stable compaction writes the row.
+constexpr int kMergeThreads = 1024;
+constexpr int kMaxSplits = 16;
+
+__device__ __forceinline__ int block_excl_scan(int x, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
+    }
+    warp_sums[lane] = wi - w;
+    if (lane == 31) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  const int r = warp_sums[warp] + incl - x;
+  total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
 
 __global__ void __launch_bounds__(kMergeThreads)
 indexer_merge_kernel(const uint64_t* __restrict__ split_out, const int* __restrict__ split_cnt,
                      int32_t* __restrict__ idx, int S, int k) {
-  __shared__ int off[33];
+  extern __shared__ uint32_t keys[];  // [S * k] score keys in union order
+  __shared__ int off[kMaxSplits + 1];
   __shared__ int hist[256];
+  __shared__ int warp_sums[33];
   __shared__ int sel_bin, kk_new, bin_count;
-  __shared__ int scan[kMergeThreads];
   const size_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const uint64_t* lists = split_out + row * S * k;
@@ -605,62 +668,109 @@ indexer_merge_kernel(const uint64_t* __restrict__ split_out, const int* __restri
   }
   __syncthreads();
   const int n = off[S];
-  auto at = [&](int e) -> unsigned long long {
+  {
     int j = 0;
-    while (off[j + 1] <= e) ++j;
-    return lists[static_cast<size_t>(j) * k + (e - off[j])];
-  };
-  unsigned long long thr = 0ull;
+    for (int e = tid; e < n; e += kMergeThreads) {
+      while (off[j + 1] <= e) ++j;
+      keys[e] = static_cast<uint32_t>(lists[static_cast<size_t>(j) * k + (e - off[j])] >> 32);
+    }
+  }
+  __syncthreads();
+  uint32_t thr = 0u;
+  int ties = 1 << 30;
   if (n > k) {
-    unsigned long long prefix = 0ull;
+    uint32_t prefix = 0u;
     int kk = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    bool exact = true;
+    for (int shift = 24; shift >= 0; shift -= 8) {
       if (tid < 256) hist[tid] = 0;
       __syncthreads();
       for (int e = tid; e < n; e += kMergeThreads) {
-        const unsigned long long v = at(e);
-        if (shift == 56 || (v >> (shift + 8)) == (prefix >> (shift + 8)))
-          atomicAdd(&hist[(v >> shift) & 255ull], 1);
+        const uint32_t key = keys[e];
+        if (shift == 24 || (key >> (shift + 8)) == (prefix >> (shift + 8)))
+          atomicAdd(&hist[(key >> shift) & 255u], 1);
       }
       __syncthreads();
-      if (tid == 0) {
-        int above = 0;
-        for (int b = 255; b >= 0; --b) {
-          if (above < kk && above + hist[b] >= kk) {
-            sel_bin = b; kk_new = kk - above; bin_count = hist[b];
-            break;
+      if (tid < 32) {
+        int loc[8];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { loc[i] = hist[tid * 8 + i]; sum += loc[i]; }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (tid + o < 32) incl += y;
+        }
+        int above = incl - sum;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (above < kk && above + loc[i] >= kk) {
+            sel_bin = tid * 8 + i;
+            kk_new = kk - above;
+            bin_count = loc[i];
           }
-          above += hist[b];
+          above += loc[i];
         }
       }
       __syncthreads();
-      prefix |= static_cast<unsigned long long>(sel_bin) << shift;
+      prefix |= static_cast<uint32_t>(sel_bin) << shift;
       kk = kk_new;
-      const bool done = bin_count == kk;
+      const bool whole_bin = bin_count == kk;
       __syncthreads();
-      if (done) break;
+      if (whole_bin) {
+        exact = false;
+        break;
+      }
     }
     thr = prefix;
+    if (exact) ties = kk;
   }
-  // stable compaction over contiguous segments
+  const bool limited = ties < (1 << 30);
+  // stable compaction over contiguous segments of the union
   const int per = (n + kMergeThreads - 1) / kMergeThreads;
-  const int e0 = tid * per, e1 = min(n, e0 + per);
-  int c = 0;
-  for (int e = e0; e < e1; ++e) c += at(e) >= thr;
-  scan[tid] = c;
-  __syncthreads();
-  for (int d = 1; d < kMergeThreads; d <<= 1) {
-    const int y = tid >= d ? scan[tid - d] : 0;
-    __syncthreads();
-    scan[tid] += y;
-    __syncthreads();
+  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+  int n_tie = 0;
+  if (limited)
+    for (int e = e0; e < e1; ++e) n_tie += keys[e] == thr;
+  int tie_total;
+  int tie_rank = block_excl_scan(n_tie, warp_sums, tie_total);
+  int n_keep = 0;
+  {
+    int tr = tie_rank;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t key = keys[e];
+      bool kp;
+      if (limited) {
+        kp = key > thr || (key == thr && tr < ties);
+        tr += key == thr;
+      } else {
+        kp = key >= thr;
+      }
+      n_keep += kp;
+    }
   }
-  int pos = scan[tid] - c;
-  const int total = scan[kMergeThreads - 1];
+  int total;
+  int pos = block_excl_scan(n_keep, warp_sums, total);
   int32_t* out = idx + row * k;
-  for (int e = e0; e < e1; ++e) {
-    const unsigned long long v = at(e);
-    if (v >= thr) out[pos++] = static_cast<int32_t>(~static_cast<uint32_t>(v & 0xffffffffull));
+  {
+    int tr = tie_rank;
+    int j = 0;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t key = keys[e];
+      bool kp;
+      if (limited) {
+        kp = key > thr || (key == thr && tr < ties);
+        tr += key == thr;
+      } else {
+        kp = key >= thr;
+      }
+      if (kp) {
+        while (off[j + 1] <= e) ++j;
+        const uint64_t v = lists[static_cast<size_t>(j) * k + (e - off[j])];
+        out[pos++] = static_cast<int32_t>(~static_cast<uint32_t>(v & 0xffffffffull));
+      }
+    }
   }
   for (int q = total + tid; q < k; q += kMergeThreads) out[q] = -1;
 }
@@ -674,7 +784,7 @@ dsa_status launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const Params&
                                             kQB * H * 4 + static_cast<int>(sizeof(EpiShared)) +
                                             (2 * C::kStages + 6) * 8 + 32);
   auto kern = indexer_topk_kernel<H, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer smem attribute: ") + cudaGetErrorString(e));
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
   e = cudaGetLastError();
@@ -701,7 +811,7 @@ IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k) {
   if (base_items < 148) {
     S = static_cast<int>(148 / base_items);
     S = std::min(S, std::max(1, max_tiles / 8));
-    S = std::min(S, 32);
+    S = std::min(S, kMaxSplits);
   }
   pl.S = S;
   const int tiles_per_split = max_tiles > 0 ? (max_tiles + S - 1) / S : 1;
@@ -759,7 +869,12 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
 #undef DSA_CASE
   if (st != DSA_OK) return st == DSA_ERR_UNSUPPORTED ? set_error(st, "indexer shape unsupported") : st;
   if (pl.S > 1) {
-    indexer_merge_kernel<<<static_cast<unsigned>(static_cast<size_t>(B) * Lq), kMergeThreads, 0, stream>>>(
+    const int msmem = pl.S * k * 4;
+    if (msmem > 48 * 1024) {
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(indexer_merge_kernel), msmem);
+      if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge smem attribute: ") + cudaGetErrorString(e));
+    }
+    indexer_merge_kernel<<<static_cast<unsigned>(static_cast<size_t>(B) * Lq), kMergeThreads, msmem, stream>>>(
         p.split_out, p.split_cnt, idx, pl.S, k);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge launch: ") + cudaGetErrorString(e));

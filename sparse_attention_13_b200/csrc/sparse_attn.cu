@@ -738,8 +738,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k;
     p.S = sp.S; p.cps = sp.cps;
     p.scale_log2 = scale * 1.4426950408889634f;
-    cudaError_t e = cudaFuncSetAttribute(mla_sparse_attn_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(mla_sparse_attn_kernel), kMlaSmem);
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla smem attribute: ") + cudaGetErrorString(e));
     mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * sp.pairs), kMlaThreads, kMlaSmem, stream>>>(tkv, p);
     e = cudaGetLastError();
@@ -755,8 +754,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
   if (n_h <= 128 && D_qk <= 128 && D_v <= 128) {
     const int smem = n_h * D_qk * 4;
     if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(simt_sparse_attn_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(simt_sparse_attn_kernel), smem);
       if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("simt smem attribute: ") + cudaGetErrorString(e));
     }
     simt_sparse_attn_kernel<<<static_cast<unsigned>(rows), kSimtThreads, smem, stream>>>(

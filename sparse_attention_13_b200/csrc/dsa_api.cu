@@ -150,9 +150,9 @@ const char* dsa_last_error(void) { return g_last_error.c_str(); }
 long long dsa_indexer_launch_count(void) { return g_indexer_launches.load(); }
 
 size_t dsa_indexer_topk_workspace(int B, int Lq, int Lk, int start_pos, int H_I, int d_I, int k) {
-  (void)H_I;
-  (void)d_I;
   if (B < 1 || Lq < 1 || k < 1 || start_pos < 0) return 0;
+  // decode rows keep one score key per cached position instead
+  if (decode_indexer_applies(Lq, Lk, start_pos, H_I, d_I)) return decode_indexer_ws_bytes(B, Lk);
   return indexer_plan(B, Lq, Lk, start_pos, std::min(k, 2048)).total_bytes;
 }
 

@@ -53,6 +53,15 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
                                int B, int Lq, int Lk, int start_pos, int H, int d, int k,
                                int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+// ---- decode indexer + top-k (decode_indexer.cu): one query row per sequence
+// against a long cache; used by indexer_topk_launch when it applies and the
+// workspace holds a row of score keys per sequence.
+bool decode_indexer_applies(int Lq, int Lk, int start_pos, int H, int d);
+size_t decode_indexer_ws_bytes(int B, int Lk);
+dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w, int B,
+                                 int Lk, int start_pos, int H, int d, int k, int32_t* idx, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream);
+
 // ---- sparse attention (sparse_attn.cu)
 size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k);
 dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,

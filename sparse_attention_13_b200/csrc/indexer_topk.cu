@@ -830,6 +830,8 @@ IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k) {
 dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
                                int B, int Lq, int Lk, int start_pos, int H, int d, int k,
                                int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (decode_indexer_applies(Lq, Lk, start_pos, H, d) && ws_bytes >= decode_indexer_ws_bytes(B, Lk))
+    return decode_indexer_launch(q_idx, k_idx, w, B, Lk, start_pos, H, d, k, idx, ws, ws_bytes, stream);
   IndexerPlan pl = indexer_plan(B, Lq, Lk, start_pos, k);
   if (ws_bytes < pl.total_bytes) return set_error(DSA_ERR_WORKSPACE, "indexer workspace too small");
   const int sms = device_sm_count();

@@ -23,6 +23,7 @@
 // threads -- race on it; issue them one after another.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "dsa_internal.h"
@@ -67,7 +68,11 @@ extern "C" dsa_status dsa_indexer_topk_noalloc(const dsa_bf16* q_idx, const dsa_
   // Size check first: reject shapes whose scratch would not fit before
   // touching the device.
   if (B >= 1 && Lq >= 1 && k >= 1 && start_pos >= 0) {
-    const size_t need = dsa_indexer_topk_workspace(B, Lq, Lk, start_pos, H_I, d_I, k);
+    // the smaller of the decode-row layout (when it applies) and the
+    // candidate-buffer layout; the launch picks whichever fits
+    size_t need = indexer_plan(B, Lq, Lk, start_pos, std::min(k, 2048)).total_bytes;
+    if (decode_indexer_applies(Lq, Lk, start_pos, H_I, d_I))
+      need = std::min(need, decode_indexer_ws_bytes(B, Lk));
     if (need > kNoAllocScratchBytes)
       return set_error(DSA_ERR_WORKSPACE,
                        "dsa_indexer_topk_noalloc: this shape needs " + std::to_string(need) +

@@ -128,3 +128,65 @@ def test_deterministic_reruns(dsa):
     a = _run(dsa, q, k, w, kk)
     b = _run(dsa, q, k, w, kk)
     np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("B,Lk,start_pos,H,d,kk", [
+    (5, 20000, 20000, 64, 128, 2048),   # one query row per sequence at t = Lk
+    (3, 9001, 7777, 32, 64, 300),       # t < Lk: the tail of the cache is not visible
+    (2, 2100, 2100, 16, 128, 2048),     # T barely above k
+    (2, 1500, 1500, 64, 64, 2048),      # T < k: every visible position, -1 padding
+    (4, 130, 1, 16, 64, 5),             # T = 1: only position 0
+    (1, 50000, 49999, 64, 128, 1),      # k = 1
+])
+def test_decode_rows_integer_exact(dsa, oracle_mod, B, Lk, start_pos, H, d, kk):
+    # Lq = 1 rows take the decode path (streamed score keys + cluster radix
+    # select); integer inputs make every score exact.
+    q, k, w = indexer_inputs_host(Lk + H + kk, B, 1, Lk, H, d)
+    got = _run(dsa, q, k, w, kk, start_pos=start_pos)
+    for b in range(B):
+        I = oracle_mod.indexer_row(q[b, 0], k[b], w[b, 0], start_pos)
+        check_topk_row(got[b, 0], oracle_mod.topk_row(I, start_pos, kk), I, kk)
+
+
+@pytest.mark.parametrize("levels", [1, 2, 5])
+def test_decode_rows_heavy_ties(dsa, oracle_mod, levels):
+    # Scores take only `levels` distinct values, so the k-th score is shared by
+    # thousands of positions spread over every CTA of the select cluster; the
+    # lower positions must win.
+    B, Lk, H, d, kk = 3, 40000, 16, 64, 2048
+    rng = np.random.default_rng(100 + levels)
+    q = np.zeros((B, 1, H, d), np.float32)
+    q[:, :, :, 0] = 1.0
+    k = np.zeros((B, Lk, d), np.float32)
+    k[:, :, 0] = rng.integers(0, levels, size=(B, Lk))
+    w = np.ones((B, 1, H), np.float32)
+    qb, kb = synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k)
+    got = _run(dsa, qb, kb, w, kk, start_pos=Lk)
+    for b in range(B):
+        I = oracle_mod.indexer_row(qb[b, 0], kb[b], w[b, 0], Lk)
+        check_topk_row(got[b, 0], oracle_mod.topk_row(I, Lk, kk), I, kk)
+
+
+def test_decode_full_size_rows(dsa, oracle_mod):
+    # B = 8 sequences at 200000 cached positions, H_I = 64, d_I = 128,
+    # k = 2048, integer inputs generated on the device; three rows checked
+    # against the oracle, all eight for shape and order.
+    import torch
+    B, Lk, H, d, kk = 8, 200000, 64, 128, 2048
+    seed, layer = 5, 3
+    qd = torch.empty((B, 1, H, d), dtype=torch.bfloat16, device="cuda")
+    kd = torch.empty((B, Lk, d), dtype=torch.bfloat16, device="cuda")
+    wd = torch.empty((B, 1, H), dtype=torch.float32, device="cuda")
+    synth.fill_cuda(qd, seed, synth.Q_IDX, synth.INT9, layer)
+    synth.fill_cuda(kd, seed, synth.K_IDX, synth.INT9, layer)
+    synth.fill_cuda(wd, seed, synth.W, synth.POW2W, layer)
+    out = dsa.indexer_topk(qd, kd, wd, kk, start_pos=Lk)
+    dsa.check_device_errors()
+    got = out.cpu().numpy()
+    assert np.all(np.diff(got[:, 0], axis=-1) > 0) and got.min() >= 0 and got.max() < Lk
+    q_host = synth.tensor(seed, synth.Q_IDX, synth.INT9, layer, (B, 1, H, d))
+    w_host = synth.tensor(seed, synth.W, synth.POW2W, layer, (B, 1, H), bf16=False)
+    for b in [0, 3, 7]:
+        k_host = synth.rows(seed, synth.K_IDX, synth.INT9, layer, (B, Lk, d), np.arange(Lk) + b * Lk)
+        I = oracle_mod.indexer_row(q_host[b, 0], k_host, w_host[b, 0], Lk)
+        check_topk_row(got[b, 0], oracle_mod.topk_row(I, Lk, kk), I, kk)

@@ -9,13 +9,17 @@
 //   decode_score_kernel  one CTA per (sequence, key range): TMA streams
 //        128-key tiles through a 6-stage ring, one thread issues a
 //        128 x H_I x d_I UMMA per tile into a 4-deep TMEM ring, four
-//        epilogue warps (thread = key) apply ReLU and w and store each score
-//        as an order-preserving 32-bit key.
+//        epilogue warps (thread = key) apply ReLU and w, store each score as
+//        an order-preserving 32-bit key and count it in a 4096-bin histogram
+//        of the key's top 12 bits (written out per CTA at the end).
 //   decode_topk_kernel   one 8-CTA cluster per sequence: each CTA holds 1/8 of
-//        the row's keys in shared memory; an MSB-first radix select (8-bit
-//        digits) sums the CTAs' histograms through distributed shared memory;
-//        keys equal to the threshold are taken in position order; each CTA
-//        then writes its selected positions at its offset in the row.
+//        the row's keys in shared memory (one bulk copy).  The score
+//        histograms give the 12-bit bin of the k-th key; keys above it are
+//        kept, keys inside it go to a short candidate list on which two more
+//        10-bit radix passes (histograms summed over the cluster through
+//        distributed shared memory) find the exact k-th key.  Kept and tied
+//        positions are marked in bitmaps, ties are granted in position order,
+//        and each CTA writes its positions at its offset in the row.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -31,9 +35,18 @@ constexpr int kDecStages = 6;
 constexpr int kDecBufs = 4;         // TMEM accumulators of 64 columns
 constexpr int kDecThreads = 192;    // 4 epilogue warps, TMA warp, MMA warp
 constexpr int kDecTmaWarp = 4, kDecMmaWarp = 5;
+constexpr int kHistBins = 4096;     // top 12 bits of the score key
+constexpr int kHistShift = 20;
 constexpr int kClusterRanks = 8;
+constexpr int kPortion = kHistBins / kClusterRanks;  // bins reduced per CTA
 constexpr int kTopkThreads = 1024;
-constexpr int kMaxSlice = 48 * 1024;  // keys per CTA slice (192 KB)
+constexpr int kMaxSlice = 40 * 1024;                  // keys per CTA slice
+constexpr int kMaxWords = kMaxSlice / 32;
+constexpr int kListCap = 4096;                        // candidates per CTA
+constexpr int kMaxScoreCtasPerRow = 160;
+constexpr int kSmemLimit = 227 * 1024;
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int H, int D>
 struct DecCfg {
@@ -42,13 +55,18 @@ struct DecCfg {
   static constexpr int kQBytes = kChunks * kQChunkBytes;
   static constexpr int kKeyChunkBytes = kTile * 128;
   static constexpr int kStageBytes = kTile * D * 2;
+  static constexpr int kQAlloc = (kQBytes + 1023) / 1024 * 1024;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmem = 1024 + kQAlloc + kDecStages * kStageBytes + kBarBytes + H * 4 + kHistBins * 4;
+  static_assert(kSmem <= kSmemLimit, "decode score kernel shared memory");
 };
 
 struct DecParams {
   const float* w;        // [B][H]
-  uint32_t* keys;        // [B][Lk] score keys
+  uint32_t* keys;        // [B][row_stride] score keys
+  int* hist;             // [B][n_split][4096] per-CTA key histograms
   unsigned int* err;
-  int B, Lk, T, n_split, split_len;
+  int B, row_stride, T, n_split, split_len;
 };
 
 template <int H, int D>
@@ -60,7 +78,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* q_smem = smem;
-  uint8_t* key_smem = q_smem + ((C::kQBytes + 1023) / 1024) * 1024;
+  uint8_t* key_smem = q_smem + C::kQAlloc;
   uint64_t* bars = reinterpret_cast<uint64_t*>(key_smem + kDecStages * C::kStageBytes);
   uint64_t* key_full = bars;
   uint64_t* key_empty = bars + kDecStages;
@@ -69,7 +87,8 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* q_full = t_empty + kDecBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* w_smem = reinterpret_cast<float*>(tmem_slot + 4);
+  float* w_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
+  int* hist_smem = reinterpret_cast<int*>(w_smem + H);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x / p.n_split;
@@ -85,6 +104,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     *abort_flag = 0;
     fence_barrier_init();
   }
+  for (int i = threadIdx.x; i < kHistBins; i += kDecThreads) hist_smem[i] = 0;
   if (threadIdx.x < H) w_smem[threadIdx.x] = p.w[static_cast<size_t>(b) * H + threadIdx.x];
   if (warp == kDecMmaWarp) {
     tmem_alloc(tmem_slot, kDecBufs * 64);
@@ -141,7 +161,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
     for (int j = 0; j < H; ++j) w[j] = w_smem[j];
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    uint32_t* out = p.keys + static_cast<size_t>(b) * p.Lk;
+    uint32_t* out = p.keys + static_cast<size_t>(b) * p.row_stride;
     for (int t = 0; t < n_tiles; ++t) {
       const int buf = t % kDecBufs;
       if (!mbar_wait(&t_full[buf], (t / kDecBufs) & 1, abort_flag)) break;
@@ -164,7 +184,11 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int j = 0; j < H; ++j) a[j & 3] = fmaf(fmaxf(__uint_as_float(v[j]), 0.f), w[j], a[j & 3]);
       const float score = (a[0] + a[1]) + (a[2] + a[3]);
       const int s = s_begin + t * kTile + warp * 32 + lane;
-      if (s < s_end) out[s] = float_key(score);
+      if (s < s_end) {
+        const uint32_t key = float_key(score);
+        out[s] = key;
+        atomicAdd(&hist_smem[key >> kHistShift], 1);
+      }
     }
   }
   tc_fence_before();
@@ -174,6 +198,9 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_after();
     tmem_dealloc(tmem, kDecBufs * 64);
   }
+  int4* hg = reinterpret_cast<int4*>(p.hist + static_cast<size_t>(blockIdx.x) * kHistBins);
+  const int4* hs = reinterpret_cast<const int4*>(hist_smem);
+  for (int i = threadIdx.x; i < kHistBins / 4; i += kDecThreads) hg[i] = hs[i];
 }
 
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
@@ -182,183 +209,288 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
-__device__ __forceinline__ int block_scan_excl(int x, int* ws, int& total) {
+// Exclusive prefix sum over the block's 1024 threads (thread order).
+__device__ __forceinline__ uint32_t block_scan_excl(uint32_t x, uint32_t* ws) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = x;
+  uint32_t incl = x;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += y;
   }
   if (lane == 31) ws[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int v = ws[lane];
-    int vi = v;
+    const uint32_t v = ws[lane];
+    uint32_t vi = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, vi, o);
+      const uint32_t y = __shfl_up_sync(0xffffffffu, vi, o);
       if (lane >= o) vi += y;
     }
     ws[lane] = vi - v;
-    if (lane == 31) ws[32] = vi;
   }
   __syncthreads();
-  const int r = ws[warp] + incl - x;
-  total = ws[32];
+  const uint32_t r = ws[warp] + incl - x;
   __syncthreads();
   return r;
 }
 
 struct TopkShared {
-  int hist[256];
-  int tot[256];
-  int scan_ws[33];
+  uint64_t list[kListCap];  // candidates: key << 32 | slice offset
+  uint32_t keep_bits[kMaxWords], tie_bits[kMaxWords];
+  int red[kPortion];        // this CTA's portion of the row's 12-bit histogram
+  int hist1[1024], hist2[1024];
+  uint32_t scan_ws[32];
+  uint64_t bar;
+  int abort_flag;
+  int portion_total, list_n;
+  int owner, owner_above;
   int sel_bin, kk_new, bin_count;
-  int n_gt, n_tie;
+  int n_keep, n_tie, cta_out, cta_tie_base, cta_keep;
 };
 
-__global__ void __cluster_dims__(kClusterRanks, 1, 1) __launch_bounds__(kTopkThreads, 1)
-decode_topk_kernel(const uint32_t* __restrict__ keys, int32_t* __restrict__ idx, int Lk, int T, int k) {
-  extern __shared__ uint32_t slice[];
-  __shared__ TopkShared sh;
-  const int tid = threadIdx.x;
-  const uint32_t rank = cluster_ctarank();
-  const size_t row = blockIdx.x / kClusterRanks;
-  const int per = (T + kClusterRanks - 1) / kClusterRanks;
-  const int lo = min(T, static_cast<int>(rank) * per);
-  const int n = min(T, lo + per) - lo;
-  const uint32_t* src = keys + row * Lk + lo;
-  for (int e = tid; e < n; e += kTopkThreads) slice[e] = src[e];
+constexpr int kTopkSharedBytes = round_up(static_cast<int>(sizeof(TopkShared)), 128);
+static_assert(kTopkSharedBytes + kMaxSlice * 4 <= kSmemLimit, "decode top-k shared memory");
+
+// Each thread holds one bin (count c, index bin); thread order is descending
+// bin order.  Records the bin that holds the kk-th largest key, given that
+// `base_above` keys lie in bins above all of this block's bins.
+__device__ __forceinline__ void pick_bin(int c, int bin, int kk, int base_above, TopkShared& sh) {
+  const int above = base_above + static_cast<int>(block_scan_excl(static_cast<uint32_t>(c), sh.scan_ws));
+  if (c > 0 && above < kk && above + c >= kk) {
+    sh.sel_bin = bin;
+    sh.kk_new = kk - above;
+    sh.bin_count = c;
+  }
   __syncthreads();
-  uint32_t thr = 0u;
-  int ties = 1 << 30;
-  if (T > k) {
-    uint32_t prefix = 0u;
-    int kk = k;
-    bool exact = true;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      if (tid < 256) sh.hist[tid] = 0;
+}
+
+__global__ void __cluster_dims__(kClusterRanks, 1, 1) __launch_bounds__(kTopkThreads, 1)
+decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hist, int n_split,
+                   int32_t* __restrict__ idx, int row_stride, int T, int k, unsigned int* err) {
+  extern __shared__ __align__(128) uint8_t topk_smem[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  uint32_t* slice = reinterpret_cast<uint32_t*>(topk_smem + kTopkSharedBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const size_t row = blockIdx.x / kClusterRanks;
+  const int per = round_up((T + kClusterRanks - 1) / kClusterRanks, 4);
+  const int lo = min(T, rank * per);
+  const int n = min(T, lo + per) - lo;
+  const int nw = (n + 31) / 32;
+
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    sh.abort_flag = 0;
+    sh.list_n = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0 && n > 0) {
+    const uint32_t bytes = static_cast<uint32_t>(round_up(n, 4)) * 4u;
+    mbar_arrive_expect_tx(&sh.bar, bytes);
+    bulk_load_g2s(slice, keys + row * row_stride + lo, bytes, &sh.bar);
+  }
+
+  // ---- 12-bit bin of the k-th largest key, from the score kernel's
+  // per-CTA histograms: CTA r sums bins [512 r, 512 r + 512) of the row
+  const bool select = T > k;
+  if (select && tid < kPortion) {
+    const int* hrow = hist + row * n_split * kHistBins + rank * kPortion + tid;
+    int sum = 0;
+    for (int s = 0; s < n_split; ++s) sum += hrow[static_cast<size_t>(s) * kHistBins];
+    sh.red[tid] = sum;
+  }
+  if (select) {
+    const uint32_t part = tid < kPortion ? static_cast<uint32_t>(sh.red[tid]) : 0u;
+    const uint32_t ex = block_scan_excl(part, sh.scan_ws);
+    if (tid == kPortion - 1) sh.portion_total = static_cast<int>(ex + part);
+  }
+  cluster_sync();  // every portion is reduced
+
+  uint32_t thr = 0u;   // keys >= thr (or > thr, when ties are limited) are kept
+  int ties = 1 << 30;  // keys == thr granted, in position order
+  bool list_mode = false;
+  uint32_t prefix = 0u;
+  int kk = k;
+  bool done = !select;
+  if (select) {
+    if (warp == 0) {
+      const int tot = lane < kClusterRanks
+                          ? static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.portion_total), lane)))
+                          : 0;
+      int above = 0;
+      for (int r = kClusterRanks - 1; r >= 0; --r) {
+        const int tr = __shfl_sync(0xffffffffu, tot, r);
+        if (above < k && above + tr >= k && lane == 0) {
+          sh.owner = r;
+          sh.owner_above = above;
+        }
+        above += tr;
+      }
+    }
+    __syncthreads();
+    const int owner = sh.owner;
+    int c = 0;
+    if (tid < kPortion)
+      c = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.red[kPortion - 1 - tid]), owner)));
+    pick_bin(c, owner * kPortion + kPortion - 1 - tid, kk, sh.owner_above, sh);
+    prefix = static_cast<uint32_t>(sh.sel_bin) << kHistShift;
+    kk = sh.kk_new;
+    if (sh.bin_count == kk) {  // the whole bin is taken
+      thr = prefix;
+      done = true;
+    } else {
+      list_mode = sh.bin_count <= kListCap;  // no CTA holds more than the bin's total
+    }
+  }
+  if (n > 0 && !mbar_wait(&sh.bar, 0, &sh.abort_flag) && lane == 0) atomicOr(err, 1u);
+
+  // ---- candidate list: keys above the bin are kept, keys in it are listed
+  if (list_mode) {
+    const uint32_t sel = prefix >> kHistShift;
+    for (int g = warp; g < nw; g += kTopkThreads / 32) {
+      const int e = g * 32 + lane;
+      const bool valid = e < n;
+      const uint32_t key = valid ? slice[e] : 0u;
+      const uint32_t top = key >> kHistShift;
+      const unsigned above = __ballot_sync(0xffffffffu, valid && top > sel);
+      const unsigned inbin = __ballot_sync(0xffffffffu, valid && top == sel);
+      int base = 0;
+      if (lane == 0) {
+        sh.keep_bits[g] = above;
+        sh.tie_bits[g] = 0u;
+        if (inbin) base = atomicAdd(&sh.list_n, __popc(inbin));
+      }
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if ((inbin >> lane) & 1u)
+        sh.list[base + __popc(inbin & lt_mask)] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(e);
+    }
+    __syncthreads();
+  }
+
+  // ---- two more radix passes (bits 19..10, then 9..0), over the list or,
+  // for a bin too full for the list, over the slice
+  if (!done) {
+    for (int pass = 0; pass < 2 && !done; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      const int hs = shift + 10;
+      int* h = pass == 0 ? sh.hist1 : sh.hist2;
+      h[tid] = 0;
       __syncthreads();
-      // warp-aggregated: scores cluster in a few bins, so one atomic per
-      // distinct bin and warp instead of one per key
-      for (int base = (tid & ~31); base < n; base += kTopkThreads) {
-        const int e = base + (tid & 31);
-        uint32_t bin = 256u;
-        if (e < n) {
+      if (list_mode) {
+        const int m = sh.list_n;
+        for (int i = tid; i < m; i += kTopkThreads) {
+          const uint32_t key = static_cast<uint32_t>(sh.list[i] >> 32);
+          if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
+        }
+      } else {
+        for (int e = tid; e < n; e += kTopkThreads) {
           const uint32_t key = slice[e];
-          if (shift == 24 || (key >> (shift + 8)) == (prefix >> (shift + 8))) bin = (key >> shift) & 255u;
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
-      }
-      cluster_sync();  // every CTA's histogram is complete
-      if (tid < 256) {
-        const uint32_t a = smem_u32(&sh.hist[tid]);
-        int sum = 0;
-#pragma unroll
-        for (int r = 0; r < kClusterRanks; ++r) sum += static_cast<int>(ld_cluster_u32(mapa_shared(a, r)));
-        sh.tot[tid] = sum;
-      }
-      __syncthreads();
-      if (tid < 32) {
-        int loc[8];
-        int sum = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { loc[i] = sh.tot[tid * 8 + i]; sum += loc[i]; }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_down_sync(0xffffffffu, incl, o);
-          if (tid + o < 32) incl += y;
-        }
-        int above = incl - sum;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (above < kk && above + loc[i] >= kk) {
-            sh.sel_bin = tid * 8 + i;
-            sh.kk_new = kk - above;
-            sh.bin_count = loc[i];
-          }
-          above += loc[i];
+          if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
         }
       }
-      cluster_sync();  // peers finished reading this CTA's histogram
+      cluster_sync();  // histograms of this pass complete (the two passes use separate buffers)
+      int c = 0;
+      const uint32_t a = smem_u32(&h[1023 - tid]);
+#pragma unroll
+      for (int r = 0; r < kClusterRanks; ++r) c += static_cast<int>(ld_cluster_u32(mapa_shared(a, r)));
+      pick_bin(c, 1023 - tid, kk, 0, sh);
       prefix |= static_cast<uint32_t>(sh.sel_bin) << shift;
       kk = sh.kk_new;
-      if (sh.bin_count == kk) {
-        exact = false;
-        break;
-      }
+      if (sh.bin_count == kk) done = true;  // the whole sub-bin is taken
     }
     thr = prefix;
-    if (exact) ties = kk;
+    if (!done) ties = kk;  // thr is the exact k-th key; kk of its copies are taken
   }
   const bool limited = ties < (1 << 30);
-  // this CTA's counts of keys above the threshold and equal to it
-  const int seg = (n + kTopkThreads - 1) / kTopkThreads;
-  const int e0 = min(n, tid * seg), e1 = min(n, e0 + seg);
-  int my_gt = 0, my_tie = 0;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t key = slice[e];
-    if (limited) {
-      my_gt += key > thr;
-      my_tie += key == thr;
-    } else {
-      my_gt += key >= thr;
+
+  // ---- keep / tie bitmaps
+  if (list_mode) {
+    const int m = sh.list_n;
+    for (int i = tid; i < m; i += kTopkThreads) {
+      const uint64_t ent = sh.list[i];
+      const uint32_t key = static_cast<uint32_t>(ent >> 32);
+      const int e = static_cast<int>(ent & 0xFFFFFFFFu);
+      if (limited ? key > thr : key >= thr) atomicOr(&sh.keep_bits[e >> 5], 1u << (e & 31));
+      else if (limited && key == thr) atomicOr(&sh.tie_bits[e >> 5], 1u << (e & 31));
+    }
+  } else {
+    for (int g = warp; g < nw; g += kTopkThreads / 32) {
+      const int e = g * 32 + lane;
+      const bool valid = e < n;
+      const uint32_t key = valid ? slice[e] : 0u;
+      const unsigned kb = __ballot_sync(0xffffffffu, valid && (limited ? key > thr : key >= thr));
+      const unsigned tb = __ballot_sync(0xffffffffu, valid && limited && key == thr);
+      if (lane == 0) { sh.keep_bits[g] = kb; sh.tie_bits[g] = tb; }
     }
   }
-  int tot_gt, tot_tie;
-  const int gt_base = block_scan_excl(my_gt, sh.scan_ws, tot_gt);
-  const int tie_base = block_scan_excl(my_tie, sh.scan_ws, tot_tie);
-  if (tid == 0) { sh.n_gt = tot_gt; sh.n_tie = tot_tie; }
-  cluster_sync();
-  // offsets of this CTA among the cluster (positions are ascending across ranks)
-  int out_base = 0, cta_tie_base = 0;
-  {
-    const uint32_t a_gt = smem_u32(&sh.n_gt), a_tie = smem_u32(&sh.n_tie);
-    int tb = 0;
-    for (uint32_t r = 0; r < rank; ++r) {
-      const int g = static_cast<int>(ld_cluster_u32(mapa_shared(a_gt, r)));
-      const int tc = static_cast<int>(ld_cluster_u32(mapa_shared(a_tie, r)));
-      const int take = limited ? max(0, min(tc, ties - tb)) : 0;
-      out_base += g + take;
-      tb += tc;
-    }
-    cta_tie_base = tb;
+  __syncthreads();
+
+  // ---- ties in position order, then the output offsets.  Thread tid owns
+  // bitmap words 2 tid and 2 tid + 1.
+  const int w0 = 2 * tid;
+  uint32_t kw[2] = {0u, 0u}, tw[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    if (w0 + j < nw) { kw[j] = sh.keep_bits[w0 + j]; tw[j] = sh.tie_bits[w0 + j]; }
+  const uint32_t nk = __popc(kw[0]) + __popc(kw[1]), nt = __popc(tw[0]) + __popc(tw[1]);
+  // keep and tie counts packed in one scan (each below 2^16 per CTA)
+  const uint32_t ex = block_scan_excl((nk << 16) | nt, sh.scan_ws);
+  if (tid == kTopkThreads - 1) {
+    sh.n_keep = static_cast<int>((ex >> 16) + nk);
+    sh.n_tie = static_cast<int>((ex & 0xFFFFu) + nt);
   }
-  // thread offsets: keys above thr, plus ties whose global rank is < ties
-  int my_take = 0;
+  cluster_sync();  // every CTA's totals are visible
+  if (warp == 0) {
+    int pk = 0, pt = 0;
+    if (lane < rank) {
+      pk = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_keep), lane)));
+      pt = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_tie), lane)));
+    }
+    int out_base = 0, tie_base = 0;
+    for (int r = 0; r < rank; ++r) {
+      const int kr = __shfl_sync(0xffffffffu, pk, r), tr = __shfl_sync(0xffffffffu, pt, r);
+      out_base += kr + (limited ? max(0, min(tr, ties - tie_base)) : 0);
+      tie_base += tr;
+    }
+    if (lane == 0) { sh.cta_out = out_base; sh.cta_tie_base = tie_base; }
+  }
+  __syncthreads();
   if (limited) {
-    const int t0 = cta_tie_base + tie_base;
-    my_take = max(0, min(my_tie, ties - t0));
-  }
-  int tot_keep;
-  const int pos0 = block_scan_excl(my_gt + my_take, sh.scan_ws, tot_keep);
-  (void)gt_base;
-  int32_t* out = idx + row * k;
-  {
-    int pos = out_base + pos0;
-    int tr = cta_tie_base + tie_base;
-    for (int e = e0; e < e1; ++e) {
-      const uint32_t key = slice[e];
-      bool kp;
-      if (limited) {
-        kp = key > thr || (key == thr && tr < ties);
-        tr += key == thr;
-      } else {
-        kp = key >= thr;
-      }
-      if (kp) {
-        if (pos < k) out[pos] = lo + e;
-        ++pos;
+    int tb = sh.cta_tie_base + static_cast<int>(ex & 0xFFFFu);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      uint32_t t = tw[j];
+      int allowed = max(0, min(__popc(t), ties - tb));
+      tb += __popc(t);
+      while (allowed-- > 0) {
+        kw[j] |= t & (0u - t);  // lowest remaining tied position
+        t &= t - 1u;
       }
     }
   }
+  const uint32_t mine = __popc(kw[0]) + __popc(kw[1]);
+  const uint32_t off = block_scan_excl(mine, sh.scan_ws);
+  if (tid == kTopkThreads - 1) sh.cta_keep = static_cast<int>(off + mine);
+  int32_t* out = idx + row * k;
+  int pos = sh.cta_out + static_cast<int>(off);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    uint32_t bits = kw[j];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < k) out[pos] = lo + (w0 + j) * 32 + bit;
+      ++pos;
+    }
+  }
+  __syncthreads();
   // padding when fewer than k positions are visible
   if (rank == kClusterRanks - 1) {
-    const int total = out_base + tot_keep;
-    for (int q = total + tid; q < k; q += kTopkThreads) out[q] = -1;
+    for (int q = sh.cta_out + sh.cta_keep + tid; q < k; q += kTopkThreads) out[q] = -1;
   }
   cluster_sync();  // no CTA leaves while peers may read its shared memory
 }
@@ -367,14 +499,23 @@ template <int H, int D>
 dsa_status launch_dec(const CUtensorMap& tq, const CUtensorMap& tk, const DecParams& p, int grid,
                       cudaStream_t stream) {
   using C = DecCfg<H, D>;
-  const int smem = 1024 + ((C::kQBytes + 1023) / 1024) * 1024 + kDecStages * C::kStageBytes + 512 + H * 4;
   auto kern = decode_score_kernel<H, D>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::kSmem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode score smem attribute: ") + cudaGetErrorString(e));
-  kern<<<grid, kDecThreads, smem, stream>>>(tq, tk, p);
+  kern<<<grid, kDecThreads, C::kSmem, stream>>>(tq, tk, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode score launch: ") + cudaGetErrorString(e));
   return DSA_OK;
+}
+
+int score_splits(int B, int T, int sms) {
+  const int tiles = (T + kTile - 1) / kTile;
+  const int per_row = std::max(1, std::min(sms, kMaxScoreCtasPerRow) / B);
+  return std::max(1, std::min(tiles, per_row));
+}
+
+size_t keys_bytes(int B, int Lk) {
+  return (static_cast<size_t>(B) * round_up(Lk, 4) * 4 + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -382,11 +523,14 @@ dsa_status launch_dec(const CUtensorMap& tq, const CUtensorMap& tk, const DecPar
 bool decode_indexer_applies(int Lq, int Lk, int start_pos, int H, int d) {
   const int T = start_pos;  // the single query row sits at t = start_pos
   return Lq == 1 && (H == 16 || H == 32 || H == 64) && (d == 64 || d == 128) && T >= 1 &&
-         (T + kClusterRanks - 1) / kClusterRanks <= kMaxSlice && Lk >= T;
+         round_up((T + kClusterRanks - 1) / kClusterRanks, 4) <= kMaxSlice && Lk >= T;
 }
 
 size_t decode_indexer_ws_bytes(int B, int Lk) {
-  return ((static_cast<size_t>(B) * Lk * 4 + 255) / 256) * 256;
+  // score keys, then per-CTA histograms for up to 160 score CTAs in all
+  // (independent of the device's SM count)
+  const size_t hist = static_cast<size_t>(B) * std::max(1, kMaxScoreCtasPerRow / B) * kHistBins * 4;
+  return keys_bytes(B, Lk) + hist;
 }
 
 dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w, int B,
@@ -396,14 +540,15 @@ dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, c
   if (ws_bytes < decode_indexer_ws_bytes(B, Lk)) return set_error(DSA_ERR_WORKSPACE, "indexer workspace too small");
   const int sms = device_sm_count();
   if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
+  const int n_split = score_splits(B, T, sms);
   const int tiles = (T + kTile - 1) / kTile;
-  const int n_split = std::max(1, std::min(tiles, sms / B > 0 ? sms / B : 1));
   DecParams p{};
   p.w = w;
   p.keys = static_cast<uint32_t*>(ws);
+  p.hist = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + keys_bytes(B, Lk));
   p.err = device_error_word();
   if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
-  p.B = B; p.Lk = Lk; p.T = T; p.n_split = n_split;
+  p.B = B; p.row_stride = round_up(Lk, 4); p.T = T; p.n_split = n_split;
   p.split_len = ((tiles + n_split - 1) / n_split) * kTile;
   CUtensorMap tq, tk;
   if (!encode_tiled_3d(&tq, q_idx, d, H, B, static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(H) * d * 2,
@@ -421,11 +566,12 @@ dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, c
   if (H == 64 && d == 64) st = launch_dec<64, 64>(tq, tk, p, grid, stream);
   if (H == 64 && d == 128) st = launch_dec<64, 128>(tq, tk, p, grid, stream);
   if (st != DSA_OK) return st;
-  const int per = (T + kClusterRanks - 1) / kClusterRanks;
-  const int tsmem = per * 4;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_topk_kernel), std::max(tsmem, 1));
+  const int per = round_up((T + kClusterRanks - 1) / kClusterRanks, 4);
+  const int tsmem = kTopkSharedBytes + per * 4;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_topk_kernel), tsmem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k smem attribute: ") + cudaGetErrorString(e));
-  decode_topk_kernel<<<B * kClusterRanks, kTopkThreads, tsmem, stream>>>(p.keys, idx, Lk, T, k);
+  decode_topk_kernel<<<B * kClusterRanks, kTopkThreads, tsmem, stream>>>(p.keys, p.hist, n_split, idx,
+                                                                         p.row_stride, T, k, p.err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k launch: ") + cudaGetErrorString(e));
   return DSA_OK;

@@ -14,12 +14,13 @@
 //        of the key's top 12 bits (written out per CTA at the end).
 //   decode_topk_kernel   one 8-CTA cluster per sequence: each CTA holds 1/8 of
 //        the row's keys in shared memory (one bulk copy).  The score
-//        histograms give the 12-bit bin of the k-th key; keys above it are
-//        kept, keys inside it go to a short candidate list on which two more
-//        10-bit radix passes (histograms summed over the cluster through
-//        distributed shared memory) find the exact k-th key.  Kept and tied
-//        positions are marked in bitmaps, ties are granted in position order,
-//        and each CTA writes its positions at its offset in the row.
+//        histograms, summed over the cluster through distributed shared
+//        memory, give the 12-bit bin of the k-th key; keys above it are kept,
+//        keys inside it go to a short candidate list.  Every CTA gathers the
+//        whole cluster's lists and finds the exact k-th key by two more 10-bit
+//        radix passes on its own.  Kept and tied positions are marked in
+//        bitmaps, ties are granted in position order, and each CTA writes its
+//        positions at its offset in the row.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -57,7 +58,7 @@ struct DecCfg {
   static constexpr int kStageBytes = kTile * D * 2;
   static constexpr int kQAlloc = (kQBytes + 1023) / 1024 * 1024;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmem = 1024 + kQAlloc + kDecStages * kStageBytes + kBarBytes + H * 4 + kHistBins * 4;
+  static constexpr int kSmem = 1024 + kQAlloc + kDecStages * kStageBytes + kBarBytes + kHistBins * 4;
   static_assert(kSmem <= kSmemLimit, "decode score kernel shared memory");
 };
 
@@ -87,8 +88,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* q_full = t_empty + kDecBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* w_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
-  int* hist_smem = reinterpret_cast<int*>(w_smem + H);
+  int* hist_smem = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x / p.n_split;
@@ -105,7 +105,6 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < kHistBins; i += kDecThreads) hist_smem[i] = 0;
-  if (threadIdx.x < H) w_smem[threadIdx.x] = p.w[static_cast<size_t>(b) * H + threadIdx.x];
   if (warp == kDecMmaWarp) {
     tmem_alloc(tmem_slot, kDecBufs * 64);
     tmem_relinquish();
@@ -114,6 +113,8 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == kDecTmaWarp) {
     if (lane == 0 && n_tiles > 0) {
@@ -159,7 +160,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // epilogue: thread = key (TMEM lane 32*warp + lane)
     float w[H];
 #pragma unroll
-    for (int j = 0; j < H; ++j) w[j] = w_smem[j];
+    for (int j = 0; j < H; ++j) w[j] = __ldg(p.w + static_cast<size_t>(b) * H + j);
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     uint32_t* out = p.keys + static_cast<size_t>(b) * p.row_stride;
     for (int t = 0; t < n_tiles; ++t) {
@@ -236,22 +237,33 @@ __device__ __forceinline__ uint32_t block_scan_excl(uint32_t x, uint32_t* ws) {
   return r;
 }
 
+__device__ __forceinline__ uint64_t ld_cluster_u64(uint32_t cluster_addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 struct TopkShared {
-  uint64_t list[kListCap];  // candidates: key << 32 | slice offset
+  uint64_t list[kListCap];  // this CTA's candidates, ascending: key << 32 | position
   uint32_t keep_bits[kMaxWords], tie_bits[kMaxWords];
   int red[kPortion];        // this CTA's portion of the row's 12-bit histogram
   int hist1[1024], hist2[1024];
   uint32_t scan_ws[32];
+  int warp_above[32], warp_inbin[32], warp_ibase[32];
+  int seg_base[kClusterRanks + 1], seg_n[kClusterRanks], seg_above[kClusterRanks];
+  int seg_gt[kClusterRanks], seg_tie[kClusterRanks];
   uint64_t bar;
   int abort_flag;
-  int portion_total, list_n;
+  int portion_total;
+  int n_above, n_inbin;     // read by the peers (list mode)
   int owner, owner_above;
   int sel_bin, kk_new, bin_count;
   int n_keep, n_tie, cta_out, cta_tie_base, cta_keep;
 };
 
 constexpr int kTopkSharedBytes = round_up(static_cast<int>(sizeof(TopkShared)), 128);
-static_assert(kTopkSharedBytes + kMaxSlice * 4 <= kSmemLimit, "decode top-k shared memory");
+static_assert(kTopkSharedBytes + kMaxSlice * 4 <= kSmemLimit && kMaxSlice * 4 >= kListCap * 8,
+              "decode top-k shared memory");
 
 // Each thread holds one bin (count c, index bin); thread order is descending
 // bin order.  Records the bin that holds the kk-th largest key, given that
@@ -266,6 +278,14 @@ __device__ __forceinline__ void pick_bin(int c, int bin, int kk, int base_above,
   __syncthreads();
 }
 
+// Selection modes, chosen identically by every CTA of the cluster:
+//   whole-bin  the 12-bit bin of the k-th key is taken entirely (or T <= k):
+//              keep every key >= the bin's lower edge;
+//   list       the bin holds at most kListCap keys in all: every CTA lists its
+//              keys in the bin, gathers the whole cluster's lists and finishes
+//              the selection locally (no further cluster barrier);
+//   slice      a bin too full for the lists (heavy ties): two more 10-bit
+//              passes over the slices with cluster-summed histograms.
 __global__ void __cluster_dims__(kClusterRanks, 1, 1) __launch_bounds__(kTopkThreads, 1)
 decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hist, int n_split,
                    int32_t* __restrict__ idx, int row_stride, int T, int k, unsigned int* err) {
@@ -284,10 +304,11 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
     sh.abort_flag = 0;
-    sh.list_n = 0;
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();
   if (tid == 0 && n > 0) {
     const uint32_t bytes = static_cast<uint32_t>(round_up(n, 4)) * 4u;
     mbar_arrive_expect_tx(&sh.bar, bytes);
@@ -299,9 +320,14 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   const bool select = T > k;
   if (select && tid < kPortion) {
     const int* hrow = hist + row * n_split * kHistBins + rank * kPortion + tid;
-    int sum = 0;
-    for (int s = 0; s < n_split; ++s) sum += hrow[static_cast<size_t>(s) * kHistBins];
-    sh.red[tid] = sum;
+    int part[4] = {0, 0, 0, 0};
+    int s = 0;
+    for (; s + 4 <= n_split; s += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) part[u] += hrow[static_cast<size_t>(s + u) * kHistBins];
+    }
+    for (; s < n_split; ++s) part[0] += hrow[static_cast<size_t>(s) * kHistBins];
+    sh.red[tid] = (part[0] + part[1]) + (part[2] + part[3]);
   }
   if (select) {
     const uint32_t part = tid < kPortion ? static_cast<uint32_t>(sh.red[tid]) : 0u;
@@ -312,10 +338,10 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
 
   uint32_t thr = 0u;   // keys >= thr (or > thr, when ties are limited) are kept
   int ties = 1 << 30;  // keys == thr granted, in position order
-  bool list_mode = false;
   uint32_t prefix = 0u;
   int kk = k;
   bool done = !select;
+  bool list_mode = false;
   if (select) {
     if (warp == 0) {
       const int tot = lane < kClusterRanks
@@ -348,85 +374,171 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   }
   if (n > 0 && !mbar_wait(&sh.bar, 0, &sh.abort_flag) && lane == 0) atomicOr(err, 1u);
 
-  // ---- candidate list: keys above the bin are kept, keys in it are listed
   if (list_mode) {
+    // ---- keys above the bin are kept; keys in it are listed in position
+    // order (warp w owns a contiguous run of 32-key groups: count, scan, write)
     const uint32_t sel = prefix >> kHistShift;
-    for (int g = warp; g < nw; g += kTopkThreads / 32) {
+    const int gpw = (nw + 31) / 32;
+    const int g_lo = min(nw, warp * gpw), g_hi = min(nw, g_lo + gpw);
+    int ca = 0, ci = 0;
+    for (int g = g_lo; g < g_hi; ++g) {
+      const int e = g * 32 + lane;
+      const bool valid = e < n;
+      const uint32_t top = (valid ? slice[e] : 0u) >> kHistShift;
+      ca += __popc(__ballot_sync(0xffffffffu, valid && top > sel));
+      ci += __popc(__ballot_sync(0xffffffffu, valid && top == sel));
+    }
+    if (lane == 0) { sh.warp_above[warp] = ca; sh.warp_inbin[warp] = ci; }
+    __syncthreads();
+    if (warp == 0) {
+      const int a = sh.warp_above[lane], i = sh.warp_inbin[lane];
+      int ai = a, ii = i;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, ai, o), yi = __shfl_up_sync(0xffffffffu, ii, o);
+        if (lane >= o) { ai += ya; ii += yi; }
+      }
+      sh.warp_ibase[lane] = ii - i;
+      if (lane == 31) { sh.n_above = ai; sh.n_inbin = ii; }
+    }
+    __syncthreads();
+    int base = sh.warp_ibase[warp];
+    for (int g = g_lo; g < g_hi; ++g) {
       const int e = g * 32 + lane;
       const bool valid = e < n;
       const uint32_t key = valid ? slice[e] : 0u;
       const uint32_t top = key >> kHistShift;
       const unsigned above = __ballot_sync(0xffffffffu, valid && top > sel);
       const unsigned inbin = __ballot_sync(0xffffffffu, valid && top == sel);
-      int base = 0;
-      if (lane == 0) {
-        sh.keep_bits[g] = above;
-        sh.tie_bits[g] = 0u;
-        if (inbin) base = atomicAdd(&sh.list_n, __popc(inbin));
-      }
-      base = __shfl_sync(0xffffffffu, base, 0);
+      if (lane == 0) { sh.keep_bits[g] = above; sh.tie_bits[g] = 0u; }
       if ((inbin >> lane) & 1u)
-        sh.list[base + __popc(inbin & lt_mask)] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(e);
+        sh.list[base + __popc(inbin & lt_mask)] = (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(lo + e);
+      base += __popc(inbin);
+    }
+  }
+  if (list_mode) cluster_sync();  // every CTA's list and counts are published
+
+  if (list_mode) {
+    // ---- gather the cluster's lists (ascending positions, rank by rank)
+    // into the slice buffer, which list mode no longer needs
+    uint64_t* all = reinterpret_cast<uint64_t*>(slice);
+    if (warp == 0) {
+      int ni = 0, na = 0;
+      if (lane < kClusterRanks) {
+        ni = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_inbin), lane)));
+        na = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_above), lane)));
+      }
+      int incl = ni;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane < kClusterRanks) {
+        sh.seg_base[lane] = incl - ni;
+        sh.seg_n[lane] = ni;
+        sh.seg_above[lane] = na;
+        sh.seg_gt[lane] = 0;
+        sh.seg_tie[lane] = 0;
+      }
+      if (lane == kClusterRanks - 1) sh.seg_base[kClusterRanks] = incl;
     }
     __syncthreads();
-  }
-
-  // ---- two more radix passes (bits 19..10, then 9..0), over the list or,
-  // for a bin too full for the list, over the slice
-  if (!done) {
+    const int m_all = sh.seg_base[kClusterRanks];
+    const uint32_t list0 = smem_u32(&sh.list[0]);
+    for (int i = tid; i < m_all; i += kTopkThreads) {
+      int r = 0;
+#pragma unroll
+      for (int q = 1; q < kClusterRanks; ++q)
+        if (i >= sh.seg_base[q]) r = q;
+      all[i] = ld_cluster_u64(mapa_shared(list0 + 8u * static_cast<uint32_t>(i - sh.seg_base[r]), r));
+    }
+    cluster_arrive();  // this CTA reads no more peer memory
+    __syncthreads();
+    // ---- the remaining 20 bits of the k-th key, over the gathered list
     for (int pass = 0; pass < 2 && !done; ++pass) {
       const int shift = pass == 0 ? 10 : 0;
       const int hs = shift + 10;
       int* h = pass == 0 ? sh.hist1 : sh.hist2;
       h[tid] = 0;
       __syncthreads();
-      if (list_mode) {
-        const int m = sh.list_n;
-        for (int i = tid; i < m; i += kTopkThreads) {
-          const uint32_t key = static_cast<uint32_t>(sh.list[i] >> 32);
-          if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
-        }
-      } else {
-        for (int e = tid; e < n; e += kTopkThreads) {
-          const uint32_t key = slice[e];
-          if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
-        }
+      for (int i = tid; i < m_all; i += kTopkThreads) {
+        const uint32_t key = static_cast<uint32_t>(all[i] >> 32);
+        if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
       }
-      cluster_sync();  // histograms of this pass complete (the two passes use separate buffers)
-      int c = 0;
-      const uint32_t a = smem_u32(&h[1023 - tid]);
-#pragma unroll
-      for (int r = 0; r < kClusterRanks; ++r) c += static_cast<int>(ld_cluster_u32(mapa_shared(a, r)));
-      pick_bin(c, 1023 - tid, kk, 0, sh);
+      __syncthreads();
+      pick_bin(h[1023 - tid], 1023 - tid, kk, 0, sh);
       prefix |= static_cast<uint32_t>(sh.sel_bin) << shift;
       kk = sh.kk_new;
       if (sh.bin_count == kk) done = true;  // the whole sub-bin is taken
     }
     thr = prefix;
-    if (!done) ties = kk;  // thr is the exact k-th key; kk of its copies are taken
-  }
-  const bool limited = ties < (1 << 30);
-
-  // ---- keep / tie bitmaps
-  if (list_mode) {
-    const int m = sh.list_n;
-    for (int i = tid; i < m; i += kTopkThreads) {
-      const uint64_t ent = sh.list[i];
+    if (!done) ties = kk;
+    const bool lim = ties < (1 << 30);
+    // per-rank counts of kept and tied candidates; this CTA's own bits
+    for (int i = tid; i < m_all; i += kTopkThreads) {
+      int r = 0;
+#pragma unroll
+      for (int q = 1; q < kClusterRanks; ++q)
+        if (i >= sh.seg_base[q]) r = q;
+      const uint64_t ent = all[i];
       const uint32_t key = static_cast<uint32_t>(ent >> 32);
-      const int e = static_cast<int>(ent & 0xFFFFFFFFu);
-      if (limited ? key > thr : key >= thr) atomicOr(&sh.keep_bits[e >> 5], 1u << (e & 31));
-      else if (limited && key == thr) atomicOr(&sh.tie_bits[e >> 5], 1u << (e & 31));
+      const bool gt = lim ? key > thr : key >= thr;
+      const bool tie = lim && key == thr;
+      if (gt) atomicAdd(&sh.seg_gt[r], 1);
+      if (tie) atomicAdd(&sh.seg_tie[r], 1);
+      if (r == rank && (gt || tie)) {
+        const int e = static_cast<int>(ent & 0xFFFFFFFFu) - lo;
+        atomicOr(gt ? &sh.keep_bits[e >> 5] : &sh.tie_bits[e >> 5], 1u << (e & 31));
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int out_base = 0, tie_base = 0;
+      for (int r = 0; r < rank; ++r) {
+        out_base += sh.seg_above[r] + sh.seg_gt[r] + (lim ? max(0, min(sh.seg_tie[r], ties - tie_base)) : 0);
+        tie_base += sh.seg_tie[r];
+      }
+      sh.cta_out = out_base;
+      sh.cta_tie_base = tie_base;
     }
   } else {
+    // ---- slice mode: two more radix passes over the slices
+    if (!done) {
+      for (int pass = 0; pass < 2 && !done; ++pass) {
+        const int shift = pass == 0 ? 10 : 0;
+        const int hs = shift + 10;
+        int* h = pass == 0 ? sh.hist1 : sh.hist2;
+        h[tid] = 0;
+        __syncthreads();
+        for (int e = tid; e < n; e += kTopkThreads) {
+          const uint32_t key = slice[e];
+          if ((key >> hs) == (prefix >> hs)) atomicAdd(&h[(key >> shift) & 1023u], 1);
+        }
+        cluster_sync();  // histograms of this pass complete (the two passes use separate buffers)
+        int c = 0;
+        const uint32_t a = smem_u32(&h[1023 - tid]);
+#pragma unroll
+        for (int r = 0; r < kClusterRanks; ++r) c += static_cast<int>(ld_cluster_u32(mapa_shared(a, r)));
+        pick_bin(c, 1023 - tid, kk, 0, sh);
+        prefix |= static_cast<uint32_t>(sh.sel_bin) << shift;
+        kk = sh.kk_new;
+        if (sh.bin_count == kk) done = true;  // the whole sub-bin is taken
+      }
+      thr = prefix;
+      if (!done) ties = kk;  // thr is the exact k-th key; kk of its copies are taken
+    }
+    const bool lim = ties < (1 << 30);
     for (int g = warp; g < nw; g += kTopkThreads / 32) {
       const int e = g * 32 + lane;
       const bool valid = e < n;
       const uint32_t key = valid ? slice[e] : 0u;
-      const unsigned kb = __ballot_sync(0xffffffffu, valid && (limited ? key > thr : key >= thr));
-      const unsigned tb = __ballot_sync(0xffffffffu, valid && limited && key == thr);
+      const unsigned kb = __ballot_sync(0xffffffffu, valid && (lim ? key > thr : key >= thr));
+      const unsigned tb = __ballot_sync(0xffffffffu, valid && lim && key == thr);
       if (lane == 0) { sh.keep_bits[g] = kb; sh.tie_bits[g] = tb; }
     }
   }
+  const bool limited = ties < (1 << 30);
   __syncthreads();
 
   // ---- ties in position order, then the output offsets.  Thread tid owns
@@ -439,24 +551,27 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   const uint32_t nk = __popc(kw[0]) + __popc(kw[1]), nt = __popc(tw[0]) + __popc(tw[1]);
   // keep and tie counts packed in one scan (each below 2^16 per CTA)
   const uint32_t ex = block_scan_excl((nk << 16) | nt, sh.scan_ws);
-  if (tid == kTopkThreads - 1) {
-    sh.n_keep = static_cast<int>((ex >> 16) + nk);
-    sh.n_tie = static_cast<int>((ex & 0xFFFFu) + nt);
-  }
-  cluster_sync();  // every CTA's totals are visible
-  if (warp == 0) {
-    int pk = 0, pt = 0;
-    if (lane < rank) {
-      pk = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_keep), lane)));
-      pt = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_tie), lane)));
+  if (!list_mode) {
+    if (tid == kTopkThreads - 1) {
+      sh.n_keep = static_cast<int>((ex >> 16) + nk);
+      sh.n_tie = static_cast<int>((ex & 0xFFFFu) + nt);
     }
-    int out_base = 0, tie_base = 0;
-    for (int r = 0; r < rank; ++r) {
-      const int kr = __shfl_sync(0xffffffffu, pk, r), tr = __shfl_sync(0xffffffffu, pt, r);
-      out_base += kr + (limited ? max(0, min(tr, ties - tie_base)) : 0);
-      tie_base += tr;
+    cluster_sync();  // every CTA's totals are visible
+    if (warp == 0) {
+      int pk = 0, pt = 0;
+      if (lane < rank) {
+        pk = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_keep), lane)));
+        pt = static_cast<int>(ld_cluster_u32(mapa_shared(smem_u32(&sh.n_tie), lane)));
+      }
+      int out_base = 0, tie_base = 0;
+      for (int r = 0; r < rank; ++r) {
+        const int kr = __shfl_sync(0xffffffffu, pk, r), tr = __shfl_sync(0xffffffffu, pt, r);
+        out_base += kr + (limited ? max(0, min(tr, ties - tie_base)) : 0);
+        tie_base += tr;
+      }
+      if (lane == 0) { sh.cta_out = out_base; sh.cta_tie_base = tie_base; }
     }
-    if (lane == 0) { sh.cta_out = out_base; sh.cta_tie_base = tie_base; }
+    cluster_arrive();  // this CTA reads no more peer memory
   }
   __syncthreads();
   if (limited) {
@@ -492,7 +607,7 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   if (rank == kClusterRanks - 1) {
     for (int q = sh.cta_out + sh.cta_keep + tid; q < k; q += kTopkThreads) out[q] = -1;
   }
-  cluster_sync();  // no CTA leaves while peers may read its shared memory
+  cluster_wait();  // no CTA leaves while peers may read its shared memory
 }
 
 template <int H, int D>
@@ -502,8 +617,8 @@ dsa_status launch_dec(const CUtensorMap& tq, const CUtensorMap& tk, const DecPar
   auto kern = decode_score_kernel<H, D>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::kSmem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode score smem attribute: ") + cudaGetErrorString(e));
-  kern<<<grid, kDecThreads, C::kSmem, stream>>>(tq, tk, p);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(grid), dim3(kDecThreads), C::kSmem, stream, tq, tk, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode score launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }
@@ -567,12 +682,13 @@ dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, c
   if (H == 64 && d == 128) st = launch_dec<64, 128>(tq, tk, p, grid, stream);
   if (st != DSA_OK) return st;
   const int per = round_up((T + kClusterRanks - 1) / kClusterRanks, 4);
-  const int tsmem = kTopkSharedBytes + per * 4;
+  const int tsmem = kTopkSharedBytes + std::max(per * 4, kListCap * 8);
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(decode_topk_kernel), tsmem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k smem attribute: ") + cudaGetErrorString(e));
-  decode_topk_kernel<<<B * kClusterRanks, kTopkThreads, tsmem, stream>>>(p.keys, p.hist, n_split, idx,
-                                                                         p.row_stride, T, k, p.err);
-  e = cudaGetLastError();
+  e = launch_pdl(decode_topk_kernel, dim3(B * kClusterRanks), dim3(kTopkThreads), tsmem, stream,
+                 static_cast<const uint32_t*>(p.keys), static_cast<const int*>(p.hist), n_split, idx,
+                 p.row_stride, T, k, p.err);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }

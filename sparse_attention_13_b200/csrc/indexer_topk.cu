@@ -351,6 +351,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
 
   int issued_tiles = 0;  // producer lane 0 only
   if (warp == kTmaWarp) {
@@ -658,6 +660,8 @@ indexer_merge_kernel(const uint64_t* __restrict__ split_out, const int* __restri
   __shared__ int hist[256];
   __shared__ int warp_sums[33];
   __shared__ int sel_bin, kk_new, bin_count;
+  pdl_trigger();
+  pdl_wait();
   const size_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const uint64_t* lists = split_out + row * S * k;
@@ -786,8 +790,8 @@ dsa_status launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const Params&
   auto kern = indexer_topk_kernel<H, D>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer smem attribute: ") + cudaGetErrorString(e));
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tq, tk, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }
@@ -876,9 +880,9 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(indexer_merge_kernel), msmem);
       if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge smem attribute: ") + cudaGetErrorString(e));
     }
-    indexer_merge_kernel<<<static_cast<unsigned>(static_cast<size_t>(B) * Lq), kMergeThreads, msmem, stream>>>(
-        p.split_out, p.split_cnt, idx, pl.S, k);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(indexer_merge_kernel, dim3(static_cast<unsigned>(static_cast<size_t>(B) * Lq)),
+                               dim3(kMergeThreads), msmem, stream, p.split_out, p.split_cnt, idx, pl.S, k);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge launch: ") + cudaGetErrorString(e));
   }
   return DSA_OK;

@@ -27,7 +27,10 @@
 //                    P as bf16 into a double-buffered K-major tile.
 //   The finished row is normalised by the softmax sum and stored as bf16.
 //   Few long rows (decode) split the index list across clusters; the
-//   partials (normalised O and log-sum-exp) are combined by mla_merge_kernel.
+//   partials (normalised O as bf16 pairs in a head-minor layout, so that the
+//   thread-per-head epilogue stores whole 128-byte lines, and the log-sum-exp)
+//   are combined by mla_merge_kernel, launched as a programmatic dependent of
+//   the attention kernel so that its launch overlaps the attention tail.
 //
 // simt_sparse_attn_kernel: plain CUDA-core kernel for small head dims
 // (D_qk, D_v <= 128, separate K and V tensors), one block per query row.
@@ -54,6 +57,8 @@ simt_sparse_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
                         int n_h, int Dqk, int Dv, int k, float scale, __nv_bfloat16* __restrict__ out,
                         float* __restrict__ lse) {
   extern __shared__ float qs[];  // [n_h][Dqk]
+  pdl_trigger();
+  pdl_wait();
   const size_t row = blockIdx.x;
   const int b = static_cast<int>(row / Lq);
   const int i = static_cast<int>(row % Lq);
@@ -126,6 +131,7 @@ struct MlaBars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
   uint64_t o_full, o_free, q_full;
+  uint64_t q0_full;  // first item: Q loaded by the sender and softmax warps together
   uint64_t x_full[2], x_free[2];
   unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
@@ -143,7 +149,7 @@ struct MlaParams {
   const int32_t* idx;       // [B*Lq][k]
   __nv_bfloat16* out;       // [B*Lq][128][512]
   float* lse;               // [B*Lq][128] or null
-  float* part_o;            // split partials [B*Lq][S][128][512] (S > 1)
+  uint32_t* part_o;         // split partials, bf16 pairs: [B*Lq][S][256 column pairs][128 heads]
   float* part_lse;          // [B*Lq][S][128]
   unsigned int* err;
   int B, Lq, Lk, start_pos, k;
@@ -209,6 +215,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     mbar_init(&bb->o_full, 1);
     mbar_init(&bb->o_free, kSoftWarps);
     mbar_init(&bb->q_full, kSendWarps);
+    mbar_init(&bb->q0_full, kSendWarps + kSoftWarps);
     bb->abort_flag = 0;
     fence_barrier_init();
   }
@@ -220,6 +227,10 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bb->tmem_slot;
+  // the next kernel may be scheduled now (it waits for this grid before
+  // touching memory); this grid waits for the previous one likewise
+  pdl_trigger();
+  pdl_wait();
 
   if (warp >= kProdWarp0 && warp < kProdWarp0 + kProdWarps) {
     // ------------------------------------------------------------ gather
@@ -242,11 +253,19 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const int r = c * kChunk + my_group * 4 + (lane & 3);
         return ((lane >> 2) < n_groups && r < it.nv) ? __ldg(irow + r) : -1;
       };
-      int s_next = fetch(it.c0);
-      for (int c = it.c0; c < it.c0 + it.n; ++c, ++g) {
+      // indices are fetched three chunks ahead (decode items are a few chunks
+      // long, so their whole index list is in flight at once)
+      const int c_end = it.c0 + it.n;
+      int f0 = fetch(it.c0);
+      int f1 = it.c0 + 1 < c_end ? fetch(it.c0 + 1) : -1;
+      int f2 = it.c0 + 2 < c_end ? fetch(it.c0 + 2) : -1;
+      for (int c = it.c0; c < c_end; ++c, ++g) {
         const int stage = g % kStages;
         const uint32_t ph = (g / kStages) & 1;
-        const int sidx = s_next;
+        const int sidx = f0;
+        f0 = f1;
+        f1 = f2;
+        f2 = c + 3 < c_end ? fetch(c + 3) : -1;
         const bool valid = sidx >= 0 && sidx < p.Lk;
         const int grow = row_base + (valid ? sidx : 0);   // padded rows read row 0 (masked later)
         const unsigned m = __ballot_sync(0xffffffffu, valid);
@@ -255,7 +274,6 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const int r1 = __shfl_sync(0xffffffffu, grow, src + 1);
         const int r2 = __shfl_sync(0xffffffffu, grow, src + 2);
         const int r3 = __shfl_sync(0xffffffffu, grow, src + 3);
-        if (c + 1 < it.c0 + it.n) s_next = fetch(c + 1);   // overlap the next chunk's index load
         const bool w = __all_sync(0xffffffffu, mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag));
         if (!w) { ok = false; break; }  // warp-uniform
         if (lane < n_groups) {
@@ -297,7 +315,10 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       for (int item = pair; item < n_items && ok; item += n_pairs) {
         const MlaItem it = mla_item(p, item);
         if (it.n == 0) continue;
-        if (!mbar_wait(&bb->q_full, it_n & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(it_n == 0 ? &bb->q0_full : &bb->q_full, it_n == 0 ? 0u : (it_n - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int c = 0; c < it.n && ok; ++c, ++g) {
           const int stage = g % kStages;
@@ -359,8 +380,11 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       if (ok) {
         const uint4* qsrc = reinterpret_cast<const uint4*>(
             p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0);
+        // the first item's blocks 1 and 2 are loaded by the softmax warps
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
+        for (int bi = 0; bi < 4; ++bi) {
+          if (it_n == 0 && (bi == 1 || bi == 2)) continue;
+          const int blk = bi;
           uint32_t r[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -381,7 +405,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(&bb->q_full);
+      if (lane == 0 && ok) mbar_arrive(it_n == 0 ? &bb->q0_full : &bb->q_full);
       for (int c = 0; c < it.n; ++c, ++g) {
         const int sb = g & 1;
         if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
@@ -450,9 +474,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       const bool partial = p.S > 1;
       if (it.n == 0) {
         if (partial) {
-          float* po = p.part_o + ((static_cast<size_t>(it.row) * p.S + it.split) * kNH + h) * kDV +
-                      rank * 256 + hf * 128;
-          for (int j = 0; j < 32; ++j) reinterpret_cast<float4*>(po)[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          uint32_t* po = p.part_o + ((static_cast<size_t>(it.row) * p.S + it.split) * 256 + rank * 128 + hf * 64) * kNH + h;
+          for (int j = 0; j < 64; ++j) po[j * kNH] = 0u;
           if (rank == 0 && hf == 0)
             p.part_lse[(static_cast<size_t>(it.row) * p.S + it.split) * kNH + h] = -INFINITY;
         } else {
@@ -461,6 +484,25 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = -INFINITY;
         }
         continue;
+      }
+      if (it_n == 0) {
+        // first item: query block 1 + hf of this head, loaded alongside the
+        // sender's blocks 0 and 3 so that the first QK starts sooner
+        if (ok) {
+          const uint4* qsrc = reinterpret_cast<const uint4*>(
+              p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0) + (1 + hf) * 8;
+          uint32_t ra[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 a = __ldg(qsrc + j);
+            ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+          }
+          tmem_st32x32(t_lane + kQCol + (1 + hf) * 32, ra);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&bb->q0_full);
       }
       // l_run: softmax denominator (fp32, before the bf16 rounding of P); each
       // half of a head keeps the sum of its own columns.
@@ -598,17 +640,19 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = lse_v;
       } else if (ok) {
         const size_t slot = static_cast<size_t>(it.row) * p.S + it.split;
-        float* po = p.part_o + (slot * kNH + h) * kDV + rank * 256 + hf * 128;
+        // column pair cp of head h at word (cp, h): a warp stores 128 contiguous bytes
+        uint32_t* po = p.part_o + (slot * 256 + rank * 128 + hf * 64) * kNH + h;
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
           uint32_t v[32];
           tmem_ld32<32>(t_lane + kOCol + hf * 128 + blk * 32, v);
           tmem_ld_wait();
-          float4* dst = reinterpret_cast<float4*>(po + blk * 32);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(v[4 * j]) * inv, __uint_as_float(v[4 * j + 1]) * inv,
-                                 __uint_as_float(v[4 * j + 2]) * inv, __uint_as_float(v[4 * j + 3]) * inv);
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * inv,
+                                                            __uint_as_float(v[2 * j + 1]) * inv);
+            po[(blk * 16 + j) * kNH] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
         }
         if (rank == 0 && hf == 0) p.part_lse[slot * kNH + h] = lse_v;
       }
@@ -631,48 +675,71 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
 }
 
 // Combines the S key-range partials of each row: out = sum_j w_j o_j with
-// w_j = exp(lse_j - LSE), LSE = log sum_j exp(lse_j).
-constexpr int kMergeHeads = 4;
-__global__ void __launch_bounds__(128)
-mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+// w_j = exp(lse_j - LSE), LSE = log sum_j exp(lse_j).  Block (row, cb) makes
+// output columns 32 cb .. 32 cb + 31 of all 128 heads: partial words are read
+// along the head (contiguous), the result is transposed in shared memory and
+// stored as 64-byte pieces of the head rows.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeCols = 32;
+constexpr int kMaxMergeSplits = 32;
+__global__ void __launch_bounds__(kMergeThreads)
+mla_merge_kernel(const uint32_t* __restrict__ part_o, const float* __restrict__ part_lse,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int S) {
+  // the partials are written by the attention grid this launch depends on
+  pdl_trigger();
+  pdl_wait();
   const size_t row = blockIdx.x;
-  const int h0 = blockIdx.y * kMergeHeads;
-  __shared__ float wgt[kMergeHeads][32];
-  __shared__ float lse_tot[kMergeHeads];
-  if (threadIdx.x < kMergeHeads) {
-    const int h = h0 + threadIdx.x;
+  const int cb = blockIdx.y;
+  __shared__ float wgt[kMaxMergeSplits][kNH];
+  __shared__ uint32_t tile[kNH][kMergeCols / 2 + 1];
+  const int t = threadIdx.x;
+  for (int e = t; e < S * kNH; e += kMergeThreads) wgt[e / kNH][e % kNH] = part_lse[row * S * kNH + e];
+  __syncthreads();
+  if (t < kNH) {
     float m = -INFINITY;
-    for (int j = 0; j < S; ++j) m = fmaxf(m, part_lse[(row * S + j) * kNH + h]);
+    for (int j = 0; j < S; ++j) m = fmaxf(m, wgt[j][t]);
     float z = 0.f;
     for (int j = 0; j < S; ++j) {
-      const float l = part_lse[(row * S + j) * kNH + h];
-      const float e = m == -INFINITY ? 0.f : __expf(l - m);
-      wgt[threadIdx.x][j] = e;
+      const float e = m == -INFINITY ? 0.f : __expf(wgt[j][t] - m);
+      wgt[j][t] = e;
       z += e;
     }
-    for (int j = 0; j < S; ++j) wgt[threadIdx.x][j] = z > 0.f ? wgt[threadIdx.x][j] / z : 0.f;
-    lse_tot[threadIdx.x] = z > 0.f ? m + __logf(z) : -INFINITY;
+    const float iz = z > 0.f ? 1.f / z : 0.f;
+    for (int j = 0; j < S; ++j) wgt[j][t] *= iz;
+    if (lse && cb == 0) lse[row * kNH + t] = z > 0.f ? m + __logf(z) : -INFINITY;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kMergeHeads * kDV / 4; e += blockDim.x) {
-    const int hh = e / (kDV / 4);
-    const int c4 = e % (kDV / 4);
-    const int h = h0 + hh;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < S; ++j) {
-      const float wj = wgt[hh][j];
-      if (wj == 0.f) continue;
-      const float4 v = reinterpret_cast<const float4*>(part_o + ((row * S + j) * kNH + h) * kDV)[c4];
-      acc.x += wj * v.x; acc.y += wj * v.y; acc.z += wj * v.z; acc.w += wj * v.w;
+  constexpr int kPairs = kMergeCols / 4;  // column pairs per thread (two threads per head)
+  const int h = t & (kNH - 1), half = t >> 7;
+  const int cp0 = cb * (kMergeCols / 2) + half * kPairs;
+  float acc[2 * kPairs];
+#pragma unroll
+  for (int i = 0; i < 2 * kPairs; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < S; ++j) {
+    const float wj = wgt[j][h];
+    const uint32_t* src = part_o + ((row * S + j) * 256 + cp0) * kNH + h;
+    uint32_t wv[kPairs];
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) wv[i] = src[i * kNH];
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+      acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
     }
-    __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y), b2 = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&a);
-    pk.y = *reinterpret_cast<uint32_t*>(&b2);
-    reinterpret_cast<uint2*>(out + (row * kNH + h) * kDV)[c4] = pk;
   }
-  if (lse && threadIdx.x < kMergeHeads) lse[row * kNH + h0 + threadIdx.x] = lse_tot[threadIdx.x];
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {
+    const __nv_bfloat162 pr = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    tile[h][half * kPairs + i] = *reinterpret_cast<const uint32_t*>(&pr);
+  }
+  __syncthreads();
+  uint32_t* orow = reinterpret_cast<uint32_t*>(out + row * kNH * kDV) + cb * (kMergeCols / 2);
+  for (int e = t; e < kNH * (kMergeCols / 2); e += kMergeThreads) {
+    const int hh = e / (kMergeCols / 2), w = e % (kMergeCols / 2);
+    orow[hh * (kDV / 2) + w] = tile[hh][w];
+  }
 }
 
 struct MlaSplit {
@@ -703,7 +770,7 @@ size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k) {
   // sized for up to 160 SMs so the requirement does not depend on the device
   const MlaSplit sp = mla_split(rows, k, 160);
   if (sp.S <= 1) return 0;
-  return static_cast<size_t>(rows) * sp.S * kNH * (kDV + 1) * sizeof(float) + 256;
+  return static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2 + 1) * 4 + 256;
 }
 
 dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
@@ -720,7 +787,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
     const MlaSplit sp = mla_split(rows, k, std::min(sms, 160));
     if (rows * sp.S > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
-    const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV + 1) * sizeof(float) : 0;
+    const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2 + 1) * 4 : 0;
     if (need > ws_bytes || (need && !ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_sparse_attn: workspace too small");
     CUtensorMap tkv;
     if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(B) * Lk,
@@ -731,8 +798,10 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     p.idx = idx;
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.lse = lse;
-    p.part_o = sp.S > 1 ? static_cast<float*>(ws) : nullptr;
-    p.part_lse = sp.S > 1 ? static_cast<float*>(ws) + static_cast<size_t>(rows) * sp.S * kNH * kDV : nullptr;
+    p.part_o = sp.S > 1 ? static_cast<uint32_t*>(ws) : nullptr;
+    p.part_lse = sp.S > 1 ? reinterpret_cast<float*>(static_cast<uint32_t*>(ws) +
+                                                     static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2))
+                          : nullptr;
     p.err = device_error_word();
     if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
     p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k;
@@ -740,13 +809,15 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(mla_sparse_attn_kernel), kMlaSmem);
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla smem attribute: ") + cudaGetErrorString(e));
-    mla_sparse_attn_kernel<<<static_cast<unsigned>(2 * sp.pairs), kMlaThreads, kMlaSmem, stream>>>(tkv, p);
-    e = cudaGetLastError();
+    e = launch_pdl(mla_sparse_attn_kernel, dim3(static_cast<unsigned>(2 * sp.pairs)), dim3(kMlaThreads), kMlaSmem,
+                   stream, tkv, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla launch: ") + cudaGetErrorString(e));
     if (sp.S > 1) {
-      mla_merge_kernel<<<dim3(static_cast<unsigned>(rows), kNH / kMergeHeads), 128, 0, stream>>>(
-          p.part_o, p.part_lse, p.out, lse, sp.S);
-      e = cudaGetLastError();
+      e = launch_pdl(mla_merge_kernel, dim3(static_cast<unsigned>(rows), kDV / kMergeCols), dim3(kMergeThreads), 0,
+                     stream, static_cast<const uint32_t*>(p.part_o), static_cast<const float*>(p.part_lse), p.out,
+                     lse, sp.S);
+      if (e == cudaSuccess) e = cudaGetLastError();
       if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla merge launch: ") + cudaGetErrorString(e));
     }
     return DSA_OK;
@@ -757,11 +828,12 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(simt_sparse_attn_kernel), smem);
       if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("simt smem attribute: ") + cudaGetErrorString(e));
     }
-    simt_sparse_attn_kernel<<<static_cast<unsigned>(rows), kSimtThreads, smem, stream>>>(
-        reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kbuf),
-        k_row_stride, reinterpret_cast<const __nv_bfloat16*>(vbuf), v_row_stride, idx, B, Lq, Lk,
-        start_pos, n_h, D_qk, D_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(simt_sparse_attn_kernel, dim3(static_cast<unsigned>(rows)), dim3(kSimtThreads), smem,
+                               stream, reinterpret_cast<const __nv_bfloat16*>(q),
+                               reinterpret_cast<const __nv_bfloat16*>(kbuf), k_row_stride,
+                               reinterpret_cast<const __nv_bfloat16*>(vbuf), v_row_stride, idx, B, Lq, Lk,
+                               start_pos, n_h, D_qk, D_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("simt attention launch: ") + cudaGetErrorString(e));
     return DSA_OK;
   }

@@ -10,7 +10,9 @@ the device; every input of the timed region is larger than L2 (126 MB), so no
 flush is needed.  A prefill step runs, per layer, the indexer (F layers) and
 the sparse attention through the C ABI with CUDA events between launches;
 the e2e figure runs the public indexcache_forward() with inputs copied from
-pinned host memory every step and the final output copied back.
+pinned host memory every step and the final output copied back.  The decode
+step is timed as replays of one CUDA graph holding the whole 48-layer step
+(per-kernel times come from separate eager steps with events).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
 Multi-GPU: launched by torchrun, one independent replica per rank (weak scaling;
@@ -336,25 +338,47 @@ def run_dsa(args):
             if events is not None:
                 events["attn"][-1][1].record(stream)
 
-    dsteps = max(args.steps, 10)
     for _ in range(max(args.warmup, 3)):
         dstep()
     barrier()
     torch.cuda.synchronize(dev)
+    # per-kernel breakdown: eager steps with events between the calls
+    dev_ev = {"idx": [], "attn": []}
+    for _ in range(3):
+        dstep(dev_ev)
+    torch.cuda.synchronize(dev)
+    d_idx_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["idx"])
+    d_attn_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["attn"])
+    # the timed decode step is one CUDA graph of the whole 48-layer step (the
+    # way a decode loop replays it); ~0.5 s of replays so the clocks are sampled
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        dstep()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dstep()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    dsa.check_device_errors()
+    dsteps = 200
+    barrier()
+    torch.cuda.synchronize(dev)
     dclocks = ClockSampler(uuid)
     dclocks.start()
-    dev_ev = {"idx": [], "attn": []}
     t0.record(stream)
     for _ in range(dsteps):
-        dstep(dev_ev)
+        graph.replay()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     dclk = dclocks.stop()
     barrier()
     dsa.check_device_errors()
     dms = max_over_ranks(t0.elapsed_time(t1) / dsteps)
-    d_idx_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["idx"])
-    d_attn_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["attn"])
+    del graph
     nFd = dpat.count("F")
     idx_bytes = B * ctx * D["d_I"] * 2 + B * D["H_I"] * D["d_I"] * 2 + B * kd * 4
     attn_bytes = B * kd * D["D_qk"] * 2 + B * D["n_h"] * (D["D_qk"] + D["D_v"]) * 2 + B * kd * 4
@@ -383,20 +407,21 @@ def run_dsa(args):
         de2e_step()
     torch.cuda.synchronize(dev)
     barrier()
+    e2e_steps = 20
     t0.record(stream)
-    for _ in range(dsteps):
+    for _ in range(e2e_steps):
         de2e_step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    de2e_ms = max_over_ranks(t0.elapsed_time(t1) / dsteps)
+    de2e_ms = max_over_ranks(t0.elapsed_time(t1) / e2e_steps)
     dh2d = sum(d_.numel() * d_.element_size() for d_, _ in hq + hqi + hw)
     result["decode"] = dict(ms_per_step=dms, idx_ms=d_idx_ms, attn_ms=d_attn_ms,
                             step_bytes=step_bytes, clocks=dclk,
                             e2e={"value": de2e_ms, "unit": "ms/step", "h2d_bytes_per_step": dh2d,
                                  "d2h_bytes_per_step": hout.numel() * 2})
-    n_merge = 1  # the split decode indexer launches a merge kernel after each F layer
-    result["decode"]["launches"] = dsteps * (nFd * (1 + n_merge) + len(dpat))
+    # per step: score + top-k kernels per F layer, attention + split merge per layer
+    result["decode"]["launches"] = dsteps * (2 * nFd + 2 * len(dpat))
     result["peaks"] = (hbm_peak, tc_peak, peak_kind)
     result["world"] = world
     if world > 1:
@@ -605,6 +630,8 @@ def main():
                              "avg_launch_ms": pf["idx_ms"]},
         "indexer_share": pf["indexer_share"],
         "decode": {"ms_per_step": dc["ms_per_step"], "higher_is_better": False,
+                   "timing": "CUDA graph of the 48-layer step, 200 replays",
+                   "gpu_launches": dc["launches"],
                    "idx_launch_ms": dc["idx_ms"], "attn_launch_ms": dc["attn_ms"],
                    "roofline": {"bound": "hbm", "achieved": dc["step_bytes"] / dc["ms_per_step"] / 1e6,
                                 "peak": hbm_peak, "unit": "GB/s",

@@ -181,6 +181,10 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Split halves of cluster_sync: arrive once this thread is done with its
 // peers' shared memory, wait before leaving.
 __device__ __forceinline__ void cluster_arrive() {

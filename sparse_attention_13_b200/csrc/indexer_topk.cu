@@ -14,7 +14,8 @@
 //            TMEM lane is one key and the ReLU/head-weighted sum over the
 //            4H columns of a query needs no cross-lane reduction.
 //   warps 0-7 epilogue: tcgen05.ld a key's H head dots per query, fold
-//            w[t,j]*max(dot,0) in fp32 (fixed head order -> deterministic),
+//            w[t,j]*max(dot,0) in fp32 (four chains over heads j mod 4 in a
+//            fixed order, the same as the decode kernel's: deterministic),
 //            pack (order-preserving score key << 32 | ~s) into one uint64 so a
 //            plain integer order is (score desc, position asc), and append the
 //            entries that beat the query's running threshold to a per-query
@@ -486,19 +487,21 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+            // heads j = 4c + r accumulate into a[r] (four independent FMA
+            // chains), combined as (a0 + a1) + (a2 + a3)
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
               const float4* w4 = reinterpret_cast<const float4*>(w_smem + (4 * h + 2 * jp + jj) * H);
-              float a = 0.f;
+              float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < H / 4; ++c) {
                 const float4 ww = w4[c];
-                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 0]), 0.f), ww.x, a);
-                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 1]), 0.f), ww.y, a);
-                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 2]), 0.f), ww.z, a);
-                a = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 3]), 0.f), ww.w, a);
+                a[0] = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 0]), 0.f), ww.x, a[0]);
+                a[1] = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 1]), 0.f), ww.y, a[1]);
+                a[2] = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 2]), 0.f), ww.z, a[2]);
+                a[3] = fmaf(fmaxf(__uint_as_float(v[jj][4 * c + 3]), 0.f), ww.w, a[3]);
               }
-              acc[jj] = a;
+              acc[jj] = (a[0] + a[1]) + (a[2] + a[3]);
             }
           } else {
             uint32_t v[2][H];
@@ -512,10 +515,10 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
               const float* wq = w_smem + (4 * h + 2 * jp + jj) * H;
-              float a = 0.f;
+              float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int c = 0; c < H; ++c) a = fmaf(fmaxf(__uint_as_float(v[jj][c]), 0.f), wq[c], a);
-              acc[jj] = a;
+              for (int c = 0; c < H; ++c) a[c & 3] = fmaf(fmaxf(__uint_as_float(v[jj][c]), 0.f), wq[c], a[c & 3]);
+              acc[jj] = (a[0] + a[1]) + (a[2] + a[3]);
             }
           }
           // candidate test and ordered append

@@ -374,8 +374,10 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     for (int item = pair; item < n_items; item += n_pairs) {
       const MlaItem it = mla_item(p, item);
       if (it.n == 0) continue;
-      // the previous item's MMAs (which read Q) are complete once its O is
-      if (it_n > 0 && ok) ok = mbar_wait(&bb->o_full, (it_n - 1) & 1, abort_flag);
+      // Q's TMEM columns (and CTA1's rope tile) are free: this warp saw the
+      // previous item's last S, so every QK of that item has completed (no
+      // later MMA of it reads Q).  The load overlaps that item's last
+      // softmax, PV and epilogue.
       tc_fence_after();
       if (ok) {
         const uint4* qsrc = reinterpret_cast<const uint4*>(
@@ -406,6 +408,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(it_n == 0 ? &bb->q0_full : &bb->q_full);
+      if (item + n_pairs < n_items) {
+        // warm L2 with this head's part of the next item's query
+        const MlaItem nx = mla_item(p, item + n_pairs);
+        const char* nq = reinterpret_cast<const char*>(p.q + (static_cast<size_t>(nx.row) * kNH + h) * kDQK + col0);
+        for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
+      }
       for (int c = 0; c < it.n; ++c, ++g) {
         const int sb = g & 1;
         if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
@@ -547,10 +555,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
           const uint32_t vm = static_cast<uint32_t>(x);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
-            lmax = fmaxf(lmax, s[j]);
-          }
+          for (int j = 0; j < 32; ++j) s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
+          // max as a tree (short dependency chains)
+          float m8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) m8[j] = fmaxf(fmaxf(s[j], s[j + 8]), fmaxf(s[j + 16], s[j + 24]));
+          lmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
         bb->red[g & 1][hf][h] = lmax;
         ok = named_bar_and(pair_bar, 64, ok);
@@ -579,18 +589,18 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           l_run *= factor;
           m_run = cmax;
         }
-        float esum = 0.f;
         uint32_t pk[16];
+        float e4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (short chains)
         const bool live = m_run != -INFINITY;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float a = live ? ex2_approx(s[2 * j] - m_run) : 0.f;
           const float bq = live ? ex2_approx(s[2 * j + 1] - m_run) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, bq);
-          esum += a + bq;
+          e4[j & 3] += a + bq;
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        l_run += esum;
+        l_run += (e4[0] + e4[1]) + (e4[2] + e4[3]);
         // P(g) overwrites the first 32 columns of S[g & 1] once the sender has
         // read them (both halves of this head read theirs before the pair barrier)
         if (ok) ok = mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag);

@@ -569,6 +569,38 @@ def kernel_case(name, seq, reps):
         idx = torch.where(r < t, pos, torch.full_like(pos, -1)).to(torch.int32)[None].expand(B, Lq, 2048).contiguous()
         out = torch.empty((B, Lq, 128, 512), dtype=bf, device=dev)
         run = lambda: dsa.sparse_attn(q, kv, kv, idx, 1 / math.sqrt(576), D_v=512, start_pos=sp, out=out)
+    elif name == "decode_step":
+        # the whole decode step (48 layers, 1/4 F, B = 8 at 200,000 cached
+        # tokens), eager, for launch lists: `reps` steps after one warm-up step
+        D = DECODE
+        B, ctx, kd = D["B"], D["ctx"], D["k"]
+        dpat = pattern_of(D["layers"], D["ratio"])
+        qi, ki, wi, qs, kvs = {}, {}, {}, [], []
+        for l, role in enumerate(dpat):
+            if role == "F":
+                qi[l] = torch.empty((B, 1, D["H_I"], D["d_I"]), dtype=bf, device=dev)
+                ki[l] = torch.empty((B, ctx, D["d_I"]), dtype=bf, device=dev)
+                wi[l] = torch.empty((B, 1, D["H_I"]), dtype=torch.float32, device=dev)
+                synth.fill_cuda(qi[l], SEED, synth.Q_IDX, synth.INT9, l)
+                synth.fill_cuda(ki[l], SEED, synth.K_IDX, synth.INT9, l)
+                synth.fill_cuda(wi[l], SEED, synth.W, synth.POW2W, l)
+            t = torch.empty((B, 1, D["n_h"], D["D_qk"]), dtype=bf, device=dev)
+            synth.fill_cuda(t, SEED, synth.Q, synth.NORMAL, l, sigma=0.5)
+            qs.append(t)
+            t = torch.empty((B, ctx, D["D_qk"]), dtype=bf, device=dev)
+            synth.fill_cuda(t, SEED, synth.KV, synth.NORMAL, l, sigma=0.5)
+            kvs.append(t)
+        dout = torch.empty((B, 1, D["n_h"], D["D_v"]), dtype=bf, device=dev)
+        didx = torch.empty((B, 1, kd), dtype=torch.int32, device=dev)
+        dws = torch.empty(max(dsa.indexer_topk_workspace(B, 1, ctx, ctx, D["H_I"], D["d_I"], kd),
+                              dsa.sparse_attn_workspace(B, 1, D["n_h"], D["D_v"], kd)), dtype=torch.uint8, device=dev)
+        scale = 1 / math.sqrt(D["D_qk"])
+
+        def run():
+            for l, role in enumerate(dpat):
+                if role == "F":
+                    dsa.indexer_topk(qi[l], ki[l], wi[l], kd, start_pos=ctx, out=didx, ws=dws)
+                dsa.sparse_attn(qs[l], kvs[l], kvs[l], didx, scale, D_v=D["D_v"], start_pos=ctx, out=dout, ws=dws)
     else:
         raise SystemExit(f"unknown kernel case {name}")
     run()
@@ -591,7 +623,8 @@ def main():
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--seq", type=int, default=0, help="override the prefill length (testing)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", default="", help="profiling: indexer|attn|decode_idx|decode_attn")
+    ap.add_argument("--kernel-case", default="",
+                    help="profiling: indexer|attn|decode_idx|decode_attn|decode_step")
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
     if args.kernel_case:

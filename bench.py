@@ -103,6 +103,24 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+def reduce_max(x, world, device):
+    """Max of a per-rank scalar over all ranks (every rank gets the result);
+    timings are reported as the slowest rank's."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms_max):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank runs its own replica)."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -165,11 +183,7 @@ def run_dsa(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     result = {}
     # ---------------------------------------------------------------- prefill
@@ -247,7 +261,7 @@ def run_dsa(args):
     attn_flops = a_units * 2 * P["n_h"] * (P["D_qk"] + P["D_v"])
     idx_flops = i_pairs * 2 * P["H_I"] * P["d_I"]
     result["prefill"] = dict(
-        ms_per_step=ms, tokens_per_s=tokens / (ms / 1e3), idx_ms=idx_ms, attn_ms=attn_ms,
+        ms_per_step=ms, tokens_per_s=job_rate(L, world, ms), idx_ms=idx_ms, attn_ms=attn_ms,
         indexer_share=nF * idx_ms / (nF * idx_ms + len(pat) * attn_ms),
         attn_tflops=attn_flops / attn_ms / 1e9, idx_tflops=idx_flops / idx_ms / 1e9,
         attn_flops=attn_flops, idx_flops=idx_flops, clocks=clk,
@@ -290,7 +304,7 @@ def run_dsa(args):
     barrier()
     dsa.check_device_errors()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    result["prefill"]["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+    result["prefill"]["e2e"] = {"value": job_rate(L, world, e2e_ms), "unit": "tokens/s",
                                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del host_in, out_h, q_idx, k_idx, w, kv, q, out, idx, ws, layers
     torch.cuda.empty_cache()

@@ -41,6 +41,7 @@ constexpr int kQB = 8;        // queries per work item
 constexpr int kTileK = 128;   // keys per tile = UMMA M
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kQPT = 16 / kEpiWarps;  // queries per epilogue thread in a 4-query half
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
@@ -200,7 +201,7 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
     int kk = k;
     bool exact = true;     // the loop ran down to a single key value
     for (int shift = 24; shift >= 0; shift -= 8) {
-      sh.hist[tid] = 0;
+      if (tid < 256) sh.hist[tid] = 0;
       named_bar_sync(kEpiBar, kEpiThreads);
 #pragma unroll
       for (int r = 0; r < kSelRows; ++r) {
@@ -443,7 +444,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else {
     // ---------------------------------------------------------- epilogue
     const int qd = warp & 3;       // TMEM lane quadrant
-    const int jp = warp >> 2;      // query pair within a half
+    const int qg = warp >> 2;      // query group within a half (kQPT queries)
     const int tid = threadIdx.x;
     uint32_t unit = 0;
     for (int round = 0;; ++round) {
@@ -473,15 +474,15 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
           const uint32_t buf = unit & 1;
           if (!mbar_wait(&tmem_full[buf], (unit >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          float acc[2];
+          float acc[kQPT];
           const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + buf * 256;
           if constexpr (H >= 32) {
-            uint32_t v[2][H];
+            uint32_t v[kQPT][H];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
+            for (int jj = 0; jj < kQPT; ++jj)
 #pragma unroll
               for (int c = 0; c < H / 32; ++c)
-                tmem_ld32<32>(t_lane + (2 * jp + jj) * H + c * 32,
+                tmem_ld32<32>(t_lane + (kQPT * qg + jj) * H + c * 32,
                               *reinterpret_cast<uint32_t(*)[32]>(&v[jj][c * 32]));
             tmem_ld_wait();
             tc_fence_before();
@@ -490,8 +491,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
             // heads j = 4c + r accumulate into a[r] (four independent FMA
             // chains), combined as (a0 + a1) + (a2 + a3)
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const float4* w4 = reinterpret_cast<const float4*>(w_smem + (4 * h + 2 * jp + jj) * H);
+            for (int jj = 0; jj < kQPT; ++jj) {
+              const float4* w4 = reinterpret_cast<const float4*>(w_smem + (4 * h + kQPT * qg + jj) * H);
               float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < H / 4; ++c) {
@@ -504,17 +505,17 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
               acc[jj] = (a[0] + a[1]) + (a[2] + a[3]);
             }
           } else {
-            uint32_t v[2][H];
+            uint32_t v[kQPT][H];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
-              tmem_ld32<H>(t_lane + (2 * jp + jj) * H, v[jj]);
+            for (int jj = 0; jj < kQPT; ++jj)
+              tmem_ld32<H>(t_lane + (kQPT * qg + jj) * H, v[jj]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_empty[buf]);
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const float* wq = w_smem + (4 * h + 2 * jp + jj) * H;
+            for (int jj = 0; jj < kQPT; ++jj) {
+              const float* wq = w_smem + (4 * h + kQPT * qg + jj) * H;
               float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < H; ++c) a[c & 3] = fmaf(fmaxf(__uint_as_float(v[jj][c]), 0.f), wq[c], a[c & 3]);
@@ -522,11 +523,11 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
           }
           // candidate test and ordered append
-          unsigned long long P[2];
-          unsigned msk[2];
+          unsigned long long P[kQPT];
+          unsigned msk[kQPT];
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int qs = 4 * h + 2 * jp + jj;
+          for (int jj = 0; jj < kQPT; ++jj) {
+            const int qs = 4 * h + kQPT * qg + jj;
             const int i = i0 + qs;
             const int T = p.start_pos + i;
             const bool valid = (i < p.Lq) && (s < T) && (s < it.s_end);
@@ -538,8 +539,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
           named_bar_sync(kEpiBar, kEpiThreads);
           bool need_sel = false;
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int qs = 4 * h + 2 * jp + jj;
+          for (int jj = 0; jj < kQPT; ++jj) {
+            const int qs = 4 * h + kQPT * qg + jj;
             const int base = es->cnt[par][qs];
             int off = base;
             for (int x = 0; x < qd; ++x) off += es->qcount[par][qs][x];

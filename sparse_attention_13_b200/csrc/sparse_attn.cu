@@ -554,9 +554,13 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           x = (x | (x >> 8)) & 0x0000FFFF0000FFFFull;
           x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
           const uint32_t vm = static_cast<uint32_t>(x);
+          if (vm != 0xFFFFFFFFu) {  // warp-uniform: rows are the same for every head
 #pragma unroll
-          for (int j = 0; j < 32; ++j) s[j] = ((vm >> j) & 1u) ? s[j] * p.scale_log2 : -INFINITY;
-          // max as a tree (short dependency chains)
+            for (int j = 0; j < 32; ++j) s[j] = ((vm >> j) & 1u) ? s[j] : -INFINITY;
+          }
+          // max of the raw scores as a tree (short dependency chains); the
+          // scale (> 0) is applied to the maximum and inside the exponent
+          // with one FMA per element
           float m8[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) m8[j] = fmaxf(fmaxf(s[j], s[j + 8]), fmaxf(s[j + 16], s[j + 24]));
@@ -565,7 +569,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         bb->red[g & 1][hf][h] = lmax;
         ok = named_bar_and(pair_bar, 64, ok);
         if (!ok) break;
-        const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]);
+        const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]) * p.scale_log2;
         if (cmax > m_run + kRescaleThresh) {
           const float factor = ex2_approx(m_run - cmax);  // 0 when m_run = -inf
           if (c > 0) {
@@ -594,8 +598,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const bool live = m_run != -INFINITY;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float a = live ? ex2_approx(s[2 * j] - m_run) : 0.f;
-          const float bq = live ? ex2_approx(s[2 * j + 1] - m_run) : 0.f;
+          const float a = live ? ex2_approx(fmaf(s[2 * j], p.scale_log2, -m_run)) : 0.f;
+          const float bq = live ? ex2_approx(fmaf(s[2 * j + 1], p.scale_log2, -m_run)) : 0.f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(a, bq);
           e4[j & 3] += a + bq;
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);

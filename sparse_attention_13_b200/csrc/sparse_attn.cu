@@ -384,9 +384,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0);
         // the first item's blocks 1 and 2 are loaded by the softmax warps
 #pragma unroll 1
-        for (int bi = 0; bi < 4; ++bi) {
-          if (it_n == 0 && (bi == 1 || bi == 2)) continue;
-          const int blk = bi;
+        for (int blk = 0; blk < 4; ++blk) {
+          if (it_n == 0 && (blk == 1 || blk == 2)) continue;
           uint32_t r[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -395,7 +394,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           }
           tmem_st32x32(t_lane + kQCol + blk * 32, r);
         }
-        if (rank == 1) {
+        if (rank == 1 && it_n > 0) {  // the first item's rope part: softmax warps
           // columns 512..575 -> 128B-swizzled K-major row h of the rope tile
           uint8_t* dst = qrope_smem + h * 128;
 #pragma unroll
@@ -408,14 +407,17 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(it_n == 0 ? &bb->q0_full : &bb->q_full);
-      if (item + n_pairs < n_items) {
-        // warm L2 with this head's part of the next item's query
-        const MlaItem nx = mla_item(p, item + n_pairs);
-        const char* nq = reinterpret_cast<const char*>(p.q + (static_cast<size_t>(nx.row) * kNH + h) * kDQK + col0);
-        for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
-      }
+      // this head's part of the next item's query, warmed into L2 a few chunks
+      // before it is loaded (earlier, the gathers would evict it again)
+      const char* nq = item + n_pairs < n_items
+                           ? reinterpret_cast<const char*>(
+                                 p.q + (static_cast<size_t>((item + n_pairs) / p.S) * kNH + h) * kDQK + col0)
+                           : nullptr;
+      const int c_pf = max(0, it.n - 4);
       for (int c = 0; c < it.n; ++c, ++g) {
         const int sb = g & 1;
+        if (c == c_pf && nq != nullptr)
+          for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
         if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
         tc_fence_after();
         uint32_t hv[32];
@@ -494,8 +496,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         continue;
       }
       if (it_n == 0) {
-        // first item: query block 1 + hf of this head, loaded alongside the
-        // sender's blocks 0 and 3 so that the first QK starts sooner
+        // first item: query block 1 + hf of this head (and, in CTA1, its rope
+        // columns), loaded alongside the sender's blocks 0 and 3 so that the
+        // first QK starts sooner
         if (ok) {
           const uint4* qsrc = reinterpret_cast<const uint4*>(
               p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0) + (1 + hf) * 8;
@@ -506,6 +509,15 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
           }
           tmem_st32x32(t_lane + kQCol + (1 + hf) * 32, ra);
+          if (rank == 1 && hf == 0) {
+            // CTA1: query columns 512..575 -> 128B-swizzled row h of the rope tile
+            uint8_t* dst = qrope_smem + h * 128;
+            const uint4* rsrc = reinterpret_cast<const uint4*>(
+                p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0) + 32;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + ((j ^ (h & 7)) << 4)) = __ldg(rsrc + j);
+            fence_proxy_async_smem();
+          }
           tmem_st_wait();
         }
         tc_fence_before();
@@ -690,11 +702,11 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
 
 // Combines the S key-range partials of each row: out = sum_j w_j o_j with
 // w_j = exp(lse_j - LSE), LSE = log sum_j exp(lse_j).  Block (row, cb) makes
-// output columns 32 cb .. 32 cb + 31 of all 128 heads: partial words are read
+// output columns 16 cb .. 16 cb + 15 of all 128 heads: partial words are read
 // along the head (contiguous), the result is transposed in shared memory and
-// stored as 64-byte pieces of the head rows.
+// stored as 32-byte pieces of the head rows.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeCols = 32;
+constexpr int kMergeCols = 16;
 constexpr int kMaxMergeSplits = 32;
 __global__ void __launch_bounds__(kMergeThreads)
 mla_merge_kernel(const uint32_t* __restrict__ part_o, const float* __restrict__ part_lse,

@@ -147,7 +147,7 @@ dsa_status indexcache_forward(const char *pattern, int n_layers,
  * without an allocator, or a path that must avoid cudaMalloc/cudaFree because
  * they can synchronise the device.  Same inputs, output and semantics as
  * dsa_indexer_topk, but the scratch lives in a fixed device array inside the
- * library of DSA_NOALLOC_SCRATCH_BYTES (48 MiB, held on every GPU that loads
+ * library of DSA_NOALLOC_SCRATCH_BYTES (72 MiB, held on every GPU that loads
  * the library until the process exits); that covers k <= 2048 for prefill and
  * decode shapes on up to 160 SMs.  Shapes needing more return
  * DSA_ERR_WORKSPACE before anything is enqueued.  The first call on a device
@@ -155,7 +155,7 @@ dsa_status indexcache_forward(const char *pattern, int n_layers,
  * All calls share the array: calls whose kernels overlap on the GPU (other
  * streams, other host threads) race on it and must be serialised.  The
  * library allocates nothing on this path. */
-#define DSA_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+#define DSA_NOALLOC_SCRATCH_BYTES (72u * 1024u * 1024u)
 dsa_status dsa_indexer_topk_noalloc(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
                                     const float *w, int B, int Lq, int Lk,
                                     int start_pos, int H_I, int d_I, int k,

@@ -19,7 +19,7 @@
 //            pack (order-preserving score key << 32 | ~s) into one uint64 so a
 //            plain integer order is (score desc, position asc), and append the
 //            entries that beat the query's running threshold to a per-query
-//            candidate buffer, in ascending s.  When a buffer passes 2k entries
+//            candidate buffer, in ascending s.  When a buffer passes 3k entries
 //            an exact radix select (8-bit digits, in registers) keeps the best k
 //            in place (stable) and raises the threshold to the k-th value.  At
 //            the end of the block a final select writes the row.
@@ -47,12 +47,12 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kEpiBar = 1;
 constexpr int kMaxK = 2048;
-constexpr int kSelRows = (2 * kMaxK + kTileK + kEpiThreads - 1) / kEpiThreads;  // 17
+constexpr int kSelRows = (3 * kMaxK + kTileK + kEpiThreads - 1) / kEpiThreads;  // 25
 constexpr int kMaxGrid = 160;
 constexpr int kTmemCols = 512;
 constexpr int kSmemBudget = 227 * 1024;
 
-__host__ __device__ constexpr int cap_for(int k) { return 2 * k + kTileK; }
+__host__ __device__ constexpr int cap_for(int k) { return 3 * k + kTileK; }
 
 template <int H, int D>
 struct Cfg {

@@ -131,7 +131,7 @@ def indexer_topk(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None, ws=No
     return out
 
 
-NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = 72 * 1024 * 1024
 
 
 def indexer_topk_noalloc(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None):

@@ -3,7 +3,7 @@
 It serves callers that cannot give the library device memory on demand --
 for example an inference engine whose allocator has already claimed all of
 HBM for its KV-cache pool, or a plain C program with no allocator of its
-own.  Its scratch is a fixed 48 MiB device array inside the library, shared
+own.  Its scratch is a fixed 72 MiB device array inside the library, shared
 by every call.  These tests call it through the C ABI twice in a row, on two
 different shapes, and require exactly the indices that the workspace-taking
 entry point dsa_indexer_topk returns for the same inputs; a shape whose

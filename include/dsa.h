@@ -165,6 +165,15 @@ dsa_status dsa_indexer_topk_noalloc(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx
  * counter; lets callers check that S layers run no indexer work). */
 long long dsa_indexer_launch_count(void);
 
+/* Self-test of failure detection (no counterpart in the pages): launches one
+ * CTA that waits on a barrier nothing ever completes, gives up after
+ * `limit_cycles` SM clock cycles (1 .. 2e9) and records the expiry in the
+ * device error word exactly as the library's kernels do when one of their
+ * bounded waits runs out.  The next dsa_check_device_errors() on `stream`
+ * then returns DSA_ERR_TIMEOUT, and the context stays usable.  Nothing traps
+ * or faults. */
+dsa_status dsa_selftest_wait_timeout(long long limit_cycles, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns DSA_ERR_TIMEOUT if any kernel's bounded wait expired since the last
  * call, DSA_ERR_CUDA on a CUDA error, DSA_OK otherwise. */

@@ -116,6 +116,24 @@ int device_sm_count() {
   return cache[dev];
 }
 
+// Self-test of the bounded-wait path: one CTA waits on an mbarrier that
+// nothing ever arrives on, gives up after `limit` cycles, and records the
+// expiry in the device error word the way every kernel's waits do.
+__global__ void selftest_wait_kernel(unsigned int* err, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const uint32_t a = smem_u32(&bar);
+  const long long t0 = clock64();
+  bool done = false;
+  while (!(done = mbar_try_wait(a, 0)) && clock64() - t0 < limit) {
+  }
+  if (!done && threadIdx.x == 0) atomicOr(err, 1u);
+}
+
 }  // namespace dsa
 
 using namespace dsa;
@@ -241,6 +259,17 @@ dsa_status indexcache_forward(const char* pattern, int n_layers, const dsa_layer
                                     d.scale, L.out, L.lse, ws, ws_bytes, stream);
     if (st != DSA_OK) return st;
   }
+  return DSA_OK;
+}
+
+dsa_status dsa_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > 2000000000ll)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_selftest_wait_timeout: limit out of range");
+  unsigned int* err = device_error_word();
+  if (!err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_cycles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("self-test launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }
 

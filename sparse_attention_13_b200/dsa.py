@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_BAD_PATTERN",
 EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
            "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
-           "dsa_indexer_topk_noalloc"]
+           "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout"]
 
 
 class DSAError(RuntimeError):
@@ -76,6 +76,8 @@ def lib():
         L.dsa_indexer_topk_noalloc.restype = I
         L.dsa_check_device_errors.argtypes = [P]
         L.dsa_check_device_errors.restype = I
+        L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
+        L.dsa_selftest_wait_timeout.restype = I
         _lib = L
     return _lib
 
@@ -216,3 +218,10 @@ def indexer_launch_count() -> int:
 
 def check_device_errors(stream=None) -> None:
     _check(lib().dsa_check_device_errors(stream if stream is not None else _stream()))
+
+
+def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Launches the library's bounded-wait self-test (a wait nothing completes,
+    abandoned after `limit_cycles`); the next check_device_errors() raises
+    DSA_ERR_TIMEOUT."""
+    _check(lib().dsa_selftest_wait_timeout(int(limit_cycles), stream if stream is not None else _stream()))

@@ -111,3 +111,10 @@ def test_workspace_sizes():
 
 def test_launch_counter_starts_at_zero_without_launches():
     assert dsa.indexer_launch_count() >= 0
+
+
+@pytest.mark.parametrize("limit", [0, -5, 3_000_000_000])
+def test_selftest_limit_validated_on_host(limit):
+    # the failure-detection self-test refuses out-of-range limits before any
+    # CUDA call
+    assert dsa.lib().dsa_selftest_wait_timeout(limit, None) == dsa.DSA_ERR_INVALID_ARG

@@ -10,7 +10,7 @@ import pytest
 
 from sparse_attention_13_b200 import synth
 
-from gpu_util import to_dev_bf16, to_dev_f32
+from gpu_util import check_topk_row, indexer_inputs_host, to_dev_bf16, to_dev_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -134,3 +134,21 @@ def test_bad_pattern_launches_nothing(dsa):
         dsa.indexcache_forward("SF", [{}, {}], dims, idx)
     assert e.value.status == dsa.DSA_ERR_BAD_PATTERN
     assert dsa.indexer_launch_count() == before
+
+
+def test_bounded_wait_expiry_reports_timeout_and_context_survives(dsa, oracle_mod):
+    # A wait that nothing completes gives up after ~1e6 cycles (about half a
+    # millisecond) and records the expiry; the host sees DSA_ERR_TIMEOUT once,
+    # the error word is cleared, and the next library call still works.
+    dsa.selftest_wait_timeout(1_000_000)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.check_device_errors()
+    assert e.value.status == dsa.DSA_ERR_TIMEOUT
+    dsa.check_device_errors()  # cleared
+    B, L, H, d, kk = 1, 300, 16, 64, 32
+    q, k, w = indexer_inputs_host(77, B, L, L, H, d)
+    got = dsa.indexer_topk(to_dev_bf16(q), to_dev_bf16(k), to_dev_f32(w), kk).cpu().numpy()
+    dsa.check_device_errors()
+    for i in (0, 31, 32, 299):
+        I = oracle_mod.indexer_row(q[0, i], k[0], w[0, i], i)
+        check_topk_row(got[0, i], oracle_mod.topk_row(I, i, kk), I, kk)

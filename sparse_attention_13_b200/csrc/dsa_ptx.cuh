@@ -103,26 +103,6 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
-                                              float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-// Asynchronous 16-byte store into a peer CTA's shared memory that signals
-// complete_tx (16 bytes) on the peer's mbarrier; needs no fence.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c,
-                                            float d, uint32_t cluster_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(cluster_addr),
-      "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
-      : "memory");
-}
 // Bulk DMA from this CTA's shared memory into a peer CTA's shared memory,
 // signalling complete_tx(bytes) on the peer's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_smem,
@@ -210,16 +190,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// 16-byte global -> shared copy (L2 only) and the mbarrier arrive that fires
-// when all of this thread's earlier cp.async copies have landed (counted
-// against the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 // Row gather: 4 rows (row0..row3) x box-width columns starting at column
 // `col` of a 2D tensor map whose box is one row high.

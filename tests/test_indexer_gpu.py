@@ -190,3 +190,26 @@ def test_decode_full_size_rows(dsa, oracle_mod):
         k_host = synth.rows(seed, synth.K_IDX, synth.INT9, layer, (B, Lk, d), np.arange(Lk) + b * Lk)
         I = oracle_mod.indexer_row(q_host[b, 0], k_host, w_host[b, 0], Lk)
         check_topk_row(got[b, 0], oracle_mod.topk_row(I, Lk, kk), I, kk)
+
+
+def test_prefill_200k_layer_sampled(dsa, oracle_mod):
+    # One F layer at the benchmark's prefill length (L = 200,000, H_I = 64,
+    # d_I = 128, k = 2048; the launch configuration bench.py times), integer
+    # inputs generated on the device; sampled rows against the oracle.
+    import torch
+    B, L, H, d, kk = 1, 200000, 64, 128, 2048
+    seed, layer = 4, 1
+    qd = torch.empty((B, L, H, d), dtype=torch.bfloat16, device="cuda")
+    kd = torch.empty((B, L, d), dtype=torch.bfloat16, device="cuda")
+    wd = torch.empty((B, L, H), dtype=torch.float32, device="cuda")
+    synth.fill_cuda(qd, seed, synth.Q_IDX, synth.INT9, layer)
+    synth.fill_cuda(kd, seed, synth.K_IDX, synth.INT9, layer)
+    synth.fill_cuda(wd, seed, synth.W, synth.POW2W, layer)
+    out = dsa.indexer_topk(qd, kd, wd, kk)
+    dsa.check_device_errors()
+    k_host = synth.tensor(seed, synth.K_IDX, synth.INT9, layer, (B, L, d))
+    for i in [1, 2048, 2049, 77777, 199999]:
+        qrow = synth.rows(seed, synth.Q_IDX, synth.INT9, layer, (B, L, H, d), np.arange(H) + i * H)
+        wrow = synth.rows(seed, synth.W, synth.POW2W, layer, (B, L, H), [i], bf16=False)[0]
+        I = oracle_mod.indexer_row(qrow, k_host[0], wrow, i)
+        check_topk_row(out[0, i].cpu().numpy(), oracle_mod.topk_row(I, i, kk), I, kk)

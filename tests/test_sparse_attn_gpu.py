@@ -207,3 +207,70 @@ def test_mla_split_rows_with_empty_splits(dsa, oracle_mod):
             o, l = oracle_mod.sparse_attn_row(q[b, i], kv[b], kv[b], idx[b, i], scale, Dv=512)
             _close(got[b, i], o)
             np.testing.assert_allclose(lse[b, i], l, rtol=0, atol=LSE_ATOL)
+
+
+def test_mla_decode_full_size_rows(dsa, oracle_mod):
+    # Decode at the benchmark's shape: 8 sequences at 200,000 cached tokens,
+    # k = 2048 selected rows each (key-range splits + merge); every row against
+    # the oracle, which sees only the selected latent rows (same sum).
+    import torch
+    B, Lk, k = 8, 200000, 2048
+    seed, layer = 21, 2
+    q = synth.tensor(seed, synth.Q, synth.NORMAL, layer, (B, 1, 128, 576), sigma=0.5)
+    kvd = torch.empty((B, Lk, 576), dtype=torch.bfloat16, device="cuda")
+    synth.fill_cuda(kvd, seed, synth.KV, synth.NORMAL, layer, sigma=0.5)
+    rng = np.random.default_rng(5)
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(B)]).astype(np.int32)
+    idx = idx[:, None, :]
+    scale = 1 / math.sqrt(576)
+    lse_t = torch.empty((B, 1, 128), dtype=torch.float32, device="cuda")
+    out = dsa.sparse_attn(to_dev_bf16(q), kvd, kvd, torch.from_numpy(idx).cuda(), scale, D_v=512,
+                          start_pos=Lk, lse=lse_t)
+    dsa.check_device_errors()
+    got, lse = out.float().cpu().numpy(), lse_t.cpu().numpy()
+    for b in range(B):
+        rows = synth.rows(seed, synth.KV, synth.NORMAL, layer, (B, Lk, 576),
+                          idx[b, 0].astype(np.uint64) + np.uint64(b * Lk), sigma=0.5)
+        o, l = oracle_mod.sparse_attn_row(q[b, 0], rows, rows, np.arange(k, dtype=np.int32), scale, Dv=512)
+        _close(got[b, 0], o)
+        np.testing.assert_allclose(lse[b, 0], l, rtol=0, atol=LSE_ATOL)
+
+
+def test_mla_prefill_200k_layer_sampled(dsa, oracle_mod):
+    # One attention layer at the benchmark's prefill length (L = 200,000, the
+    # launch configuration bench.py times); every row gets a valid index set,
+    # sampled rows a seeded random one checked against the oracle.
+    import torch
+    B, L, k = 1, 200000, 2048
+    seed, layer = 23, 0
+    qd = torch.empty((B, L, 128, 576), dtype=torch.bfloat16, device="cuda")
+    kvd = torch.empty((B, L, 576), dtype=torch.bfloat16, device="cuda")
+    synth.fill_cuda(qd, seed, synth.Q, synth.NORMAL, layer, sigma=0.5)
+    synth.fill_cuda(kvd, seed, synth.KV, synth.NORMAL, layer, sigma=0.5)
+    idx = torch.empty((B, L, k), dtype=torch.int32, device="cuda")
+    r = torch.arange(k, device="cuda", dtype=torch.int32)[None, :]
+    for t0 in range(0, L, 20000):  # in slabs to bound the temporaries
+        t = torch.arange(t0, min(L, t0 + 20000), device="cuda", dtype=torch.int32)[:, None]
+        idx[0, t0:t0 + t.shape[0]] = torch.where(r < t, (t - 1 - r) % torch.clamp(t, min=1), torch.full_like(r, -1))
+    rows = [0, 1, 2047, 2048, 99999, 150001, 199999]
+    rng = np.random.default_rng(29)
+    sel = {}
+    for i in rows:
+        n = min(i, k)
+        s = np.sort(rng.choice(i, size=n, replace=False)).astype(np.int32) if n else np.zeros(0, np.int32)
+        row = -np.ones(k, np.int32)
+        row[:n] = s
+        sel[i] = row
+        idx[0, i] = torch.from_numpy(row).cuda()
+    scale = 1 / math.sqrt(576)
+    out = dsa.sparse_attn(qd, kvd, kvd, idx, scale, D_v=512)
+    dsa.check_device_errors()
+    for i in rows:
+        n = min(i, k)
+        qrow = synth.rows(seed, synth.Q, synth.NORMAL, layer, (B, L, 128, 576), np.arange(128) + 128 * i, sigma=0.5)
+        if n == 0:
+            assert torch.all(out[0, i] == 0)
+            continue
+        krows = synth.rows(seed, synth.KV, synth.NORMAL, layer, (B, L, 576), sel[i][:n].astype(np.uint64), sigma=0.5)
+        o, _ = oracle_mod.sparse_attn_row(qrow, krows, krows, np.arange(n, dtype=np.int32), scale, Dv=512)
+        _close(out[0, i].float().cpu().numpy(), o)

@@ -23,8 +23,10 @@
 //            an exact radix select (8-bit digits, in registers) keeps the best k
 //            in place (stable) and raises the threshold to the k-th value.  At
 //            the end of the block a final select writes the row.
-// Long rows in tiny grids (decode) split the key range across CTAs; each
-// split keeps its own top-k and a merge kernel selects the final k.
+// Few query blocks over long key ranges (short continuation chunks; single
+// rows go to decode_indexer.cu where its shapes apply) split the key range
+// across CTAs; each split keeps its own top-k and a merge kernel selects the
+// final k.
 #include <cuda_bf16.h>
 
 #include <algorithm>

@@ -10,7 +10,9 @@ the device; every input of the timed region is larger than L2 (126 MB), so no
 flush is needed.  A prefill step runs, per layer, the indexer (F layers) and
 the sparse attention through the C ABI with CUDA events between launches;
 the e2e figure runs the public indexcache_forward() with inputs copied from
-pinned host memory every step and the final output copied back.  The decode
+pinned host memory every step and the final output copied back (double
+buffered on the device, so that one step's copies overlap the neighbouring
+steps' compute; every copy stays inside the timed region).  The decode
 step is timed as replays of one CUDA graph holding the whole 48-layer step
 (per-kernel times come from separate eager steps with events).
 
@@ -119,6 +121,58 @@ def job_rate(units_per_rank, world, ms_max):
     """Whole-job throughput: the units all ranks processed over the slowest
     rank's time (weak scaling: every rank runs its own replica)."""
     return units_per_rank * world / (ms_max / 1e3)
+
+
+def pipelined_e2e(torch, dev, stream, h2d_pairs, forward, d2h_pairs, steps):
+    """End-to-end steps with host buffers, double-buffered on the device.
+
+    Step i computes on device buffer set i % 2 (forward(set) enqueues it on
+    `stream`) while a copy stream loads step i + 1's inputs from pinned host
+    memory into the other set, and a third stream copies step i - 1's result
+    back to the host.  Every step's host-to-device inputs and device-to-host
+    result are inside the timed region, which ends when the last result is on
+    the host.  h2d_pairs[set] and d2h_pairs[set] are lists of (device tensor,
+    pinned host tensor).  Returns milliseconds per step."""
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    s_in.wait_event(t0)
+    s_out.wait_event(t0)
+    h2d_done, comp_done, d2h_done = [None, None], [None, None], [None, None]
+
+    def load(b):
+        with torch.cuda.stream(s_in):
+            if comp_done[b] is not None:
+                s_in.wait_event(comp_done[b])  # the step that last used set b is done
+            for d, h in h2d_pairs[b]:
+                d.copy_(h, non_blocking=True)
+            h2d_done[b] = torch.cuda.Event()
+            h2d_done[b].record(s_in)
+
+    load(0)
+    for i in range(steps):
+        b, nb = i % 2, (i + 1) % 2
+        if i + 1 < steps:
+            load(nb)
+        stream.wait_event(h2d_done[b])
+        if d2h_done[b] is not None:
+            stream.wait_event(d2h_done[b])  # set b's previous result has been read back
+        forward(b)
+        comp_done[b] = torch.cuda.Event()
+        comp_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            for d, h in d2h_pairs[b]:
+                h.copy_(d, non_blocking=True)
+            d2h_done[b] = torch.cuda.Event()
+            d2h_done[b].record(s_out)
+    for ev in d2h_done:
+        if ev is not None:
+            stream.wait_event(ev)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1) / steps
 
 
 def measured_peaks():
@@ -278,35 +332,35 @@ def run_dsa(args):
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     h2d = sum(d.numel() * d.element_size() for d, _ in host_in)
     d2h = out.numel() * out.element_size()
-    layers = []
-    for l, role in enumerate(pat):
-        L_ = dict(q=q, kbuf=kv[l], vbuf=kv[l], out=out)
-        if role == "F":
-            L_.update(q_idx=q_idx[l], k_idx=k_idx[l], w=w[l])
-        layers.append(L_)
+    # a second device set of every input and of the output (double buffering)
+    set_dev = [[d for d, _ in host_in], [torch.empty_like(d) for d, _ in host_in]]
+    set_out = [out, torch.empty_like(out)]
 
-    def e2e_step():
-        for d, h in host_in:
-            d.copy_(h, non_blocking=True)
-        dsa.indexcache_forward(pat, layers, dims, idx, ws=ws)
-        out_h.copy_(out, non_blocking=True)
+    def layers_of(b):
+        dmap = {id(d0): d1 for d0, d1 in zip(set_dev[0], set_dev[b])}
+        res = []
+        for l, role in enumerate(pat):
+            L_ = dict(q=dmap[id(q)], kbuf=dmap[id(kv[l])], vbuf=dmap[id(kv[l])], out=set_out[b])
+            if role == "F":
+                L_.update(q_idx=dmap[id(q_idx[l])], k_idx=dmap[id(k_idx[l])], w=dmap[id(w[l])])
+            res.append(L_)
+        return res
 
-    for _ in range(args.warmup):
-        e2e_step()
+    set_layers = [layers_of(0), layers_of(1)]
+    h2d_pairs = [[(d, h) for d, (_, h) in zip(set_dev[b], host_in)] for b in range(2)]
+    d2h_pairs = [[(set_out[b], out_h)] for b in range(2)]
+
+    def e2e_forward(b):
+        dsa.indexcache_forward(pat, set_layers[b], dims, idx, ws=ws)
+
+    pipelined_e2e(torch, dev, stream, h2d_pairs, e2e_forward, d2h_pairs, args.warmup)
     barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(pipelined_e2e(torch, dev, stream, h2d_pairs, e2e_forward, d2h_pairs, args.steps))
     barrier()
     dsa.check_device_errors()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     result["prefill"]["e2e"] = {"value": job_rate(L, world, e2e_ms), "unit": "tokens/s",
                                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del host_in, out_h, q_idx, k_idx, w, kv, q, out, idx, ws, layers
+    del host_in, out_h, q_idx, k_idx, w, kv, q, out, idx, ws, set_dev, set_out, set_layers, h2d_pairs, d2h_pairs
     torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- decode
@@ -398,37 +452,38 @@ def run_dsa(args):
     attn_bytes = B * kd * D["D_qk"] * 2 + B * D["n_h"] * (D["D_qk"] + D["D_v"]) * 2 + B * kd * 4
     step_bytes = nFd * idx_bytes + len(dpat) * attn_bytes
     # e2e: new query tokens in, final output out; caches stay resident
-    dlayers = []
     hq = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in dq]
     hqi = [(dq_idx[l], torch.empty(dq_idx[l].shape, dtype=bf, pin_memory=True)) for l in sorted(dq_idx)]
     hw = [(dw[l], torch.empty(dw[l].shape, dtype=f32, pin_memory=True)) for l in sorted(dw)]
     for d_, h_ in hq + hqi + hw:
         h_.copy_(d_)
     hout = torch.empty(dout.shape, dtype=bf, pin_memory=True)
-    for l, role in enumerate(dpat):
-        L_ = dict(q=dq[l], kbuf=dkv[l], vbuf=dkv[l], out=dout)
-        if role == "F":
-            L_.update(q_idx=dq_idx[l], k_idx=dk_idx[l], w=dw[l])
-        dlayers.append(L_)
+    pairs0 = hq + hqi + hw
+    dset = [[d_ for d_, _ in pairs0], [torch.empty_like(d_) for d_, _ in pairs0]]
+    dset_out = [dout, torch.empty_like(dout)]
 
-    def de2e_step():
-        for d_, h_ in hq + hqi + hw:
-            d_.copy_(h_, non_blocking=True)
-        dsa.indexcache_forward(dpat, dlayers, ddims, didx, ws=dws)
-        hout.copy_(dout, non_blocking=True)
+    def dlayers_of(b):
+        dmap = {id(d0): d1 for d0, d1 in zip(dset[0], dset[b])}
+        res = []
+        for l, role in enumerate(dpat):
+            L_ = dict(q=dmap[id(dq[l])], kbuf=dkv[l], vbuf=dkv[l], out=dset_out[b])
+            if role == "F":
+                L_.update(q_idx=dmap[id(dq_idx[l])], k_idx=dk_idx[l], w=dmap[id(dw[l])])
+            res.append(L_)
+        return res
 
-    for _ in range(3):
-        de2e_step()
-    torch.cuda.synchronize(dev)
+    dset_layers = [dlayers_of(0), dlayers_of(1)]
+    dh2d_pairs = [[(d_, h_) for d_, (_, h_) in zip(dset[b], pairs0)] for b in range(2)]
+    dd2h_pairs = [[(dset_out[b], hout)] for b in range(2)]
+
+    def de2e_forward(b):
+        dsa.indexcache_forward(dpat, dset_layers[b], ddims, didx, ws=dws)
+
+    pipelined_e2e(torch, dev, stream, dh2d_pairs, de2e_forward, dd2h_pairs, 3)
     barrier()
-    e2e_steps = 20
-    t0.record(stream)
-    for _ in range(e2e_steps):
-        de2e_step()
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
+    de2e_ms = max_over_ranks(pipelined_e2e(torch, dev, stream, dh2d_pairs, de2e_forward, dd2h_pairs, 20))
     barrier()
-    de2e_ms = max_over_ranks(t0.elapsed_time(t1) / e2e_steps)
+    dsa.check_device_errors()
     dh2d = sum(d_.numel() * d_.element_size() for d_, _ in hq + hqi + hw)
     result["decode"] = dict(ms_per_step=dms, idx_ms=d_idx_ms, attn_ms=d_attn_ms,
                             step_bytes=step_bytes, clocks=dclk,

@@ -213,3 +213,26 @@ def test_prefill_200k_layer_sampled(dsa, oracle_mod):
         wrow = synth.rows(seed, synth.W, synth.POW2W, layer, (B, L, H), [i], bf16=False)[0]
         I = oracle_mod.indexer_row(qrow, k_host[0], wrow, i)
         check_topk_row(out[0, i].cpu().numpy(), oracle_mod.topk_row(I, i, kk), I, kk)
+
+
+@pytest.mark.parametrize("T", [327680, 327681])
+def test_decode_rows_at_the_slice_limit(dsa, oracle_mod, T):
+    # The decode kernels hold 1/8 of a row's score keys per CTA (at most 40,960
+    # keys each, i.e. T <= 327,680); one more key takes the split prefill path.
+    # Both sides of the limit must give the oracle's rows.
+    import torch
+    B, H, d, kk = 1, 16, 64, 2048
+    seed, layer = 8, 0
+    qd = torch.empty((B, 1, H, d), dtype=torch.bfloat16, device="cuda")
+    kd = torch.empty((B, T, d), dtype=torch.bfloat16, device="cuda")
+    wd = torch.empty((B, 1, H), dtype=torch.float32, device="cuda")
+    synth.fill_cuda(qd, seed, synth.Q_IDX, synth.INT9, layer)
+    synth.fill_cuda(kd, seed, synth.K_IDX, synth.INT9, layer)
+    synth.fill_cuda(wd, seed, synth.W, synth.POW2W, layer)
+    out = dsa.indexer_topk(qd, kd, wd, kk, start_pos=T)
+    dsa.check_device_errors()
+    q_host = synth.tensor(seed, synth.Q_IDX, synth.INT9, layer, (B, 1, H, d))
+    w_host = synth.tensor(seed, synth.W, synth.POW2W, layer, (B, 1, H), bf16=False)
+    k_host = synth.tensor(seed, synth.K_IDX, synth.INT9, layer, (B, T, d))
+    I = oracle_mod.indexer_row(q_host[0, 0], k_host[0], w_host[0, 0], T)
+    check_topk_row(out[0, 0].cpu().numpy(), oracle_mod.topk_row(I, T, kk), I, kk)

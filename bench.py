@@ -43,6 +43,17 @@ DECODE = dict(B=8, ctx=200000, layers=48, ratio=4, H_I=64, d_I=128, k=2048, n_h=
 SEED = 1234
 
 
+WORKLOAD = ("prefill: B=1, L=200000, 16 layers FSSS x4 (1/4 F), H_I=64 d_I=128 k=2048, MLA 128 heads "
+            "576/512; decode: B=8, ctx 200000, 48 layers 1/4 F")
+
+
+def config_of(world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": WORKLOAD, "global_batch": world, "seq_len": PREFILL["L"],
+            "parallelism": f"dp{world} (independent replicas)",
+            "l2": "inputs larger than L2 (126 MB) every step; no flush"}
+
+
 def pattern_of(layers, ratio):
     return "".join("F" if l % ratio == 0 else "S" for l in range(layers))
 
@@ -597,11 +608,11 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"prefill L={P['L']}, 16 layers FSSS x4, k=2048 (CPU oracle sample)",
-                       "global_batch": 1, "seq_len": P["L"], "parallelism": "single host thread"},
+            "config": config_of(1),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "per step: 1 indexer row at t = L/2 and 1 attention row, "
-                                       "extrapolated to the 16-layer stack"},
+                             "sample": f"per step: 1 indexer row at t = L/2 (the mean causal row) and "
+                                       f"1 attention row of the L = {P['L']} prefill stack, single host "
+                                       f"thread, extrapolated to the 16-layer stack (prefill metric only)"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -717,11 +728,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "prefill: B=1, L=200000, 16 layers FSSS x4 (1/4 F), H_I=64 d_I=128 "
-                               "k=2048, MLA 128 heads 576/512; decode: B=8, ctx 200000, 48 layers "
-                               "1/4 F", "global_batch": world, "seq_len": PREFILL["L"],
-                   "parallelism": f"dp{world} (independent replicas)",
-                   "l2": "inputs larger than L2 (126 MB) every step; no flush"},
+        "config": config_of(world),
         "roofline": {"bound": "tensor", "kernel": "mla_sparse_attn", "achieved": pf["attn_tflops"],
                      "peak": tc_peak, "unit": "TFLOP/s", "frac": pf["attn_tflops"] / tc_peak,
                      "traffic": attn_tr, "peak_kind": f"{peak_kind} bf16 sustained",

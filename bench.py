@@ -608,7 +608,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": config_of(1),
+            "config": config_of(args.gpus),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"per step: 1 indexer row at t = L/2 (the mean causal row) and "
                                        f"1 attention row of the L = {P['L']} prefill stack, single host "

@@ -148,8 +148,9 @@ dsa_status indexcache_forward(const char *pattern, int n_layers,
  * they can synchronise the device.  Same inputs, output and semantics as
  * dsa_indexer_topk, but the scratch lives in a fixed device array inside the
  * library of DSA_NOALLOC_SCRATCH_BYTES (72 MiB, held on every GPU that loads
- * the library until the process exits); that covers k <= 2048 for prefill and
- * decode shapes on up to 160 SMs.  Shapes needing more return
+ * the library until the process exits); that covers k <= 2048 for prefill
+ * shapes on up to 160 SMs and decode rows (Lq = 1) up to B * Lk of about
+ * 18 million cached positions.  Shapes needing more return
  * DSA_ERR_WORKSPACE before anything is enqueued.  The first call on a device
  * looks up the array's device address (make it before any stream capture).
  * All calls share the array: calls whose kernels overlap on the GPU (other

@@ -166,6 +166,16 @@ dsa_status dsa_indexer_topk_noalloc(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx
  * counter; lets callers check that S layers run no indexer work). */
 long long dsa_indexer_launch_count(void);
 
+/* Validation of index rows (a debugging aid; the pages describe none):
+ * counts the rows of idx [B, Lq, k] (device) that are not in the canonical
+ * form dsa_indexer_topk writes -- for row i at t = start_pos + i, the first
+ * min(t, k) entries strictly ascending in [0, t) ([IDX] §4: S_t is a subset
+ * of {s : 0 <= s < t}), then -1 -- and writes the count to *bad_rows (one
+ * device int, overwritten; read it after the stream completes).  Reads idx
+ * only; allocates nothing. */
+dsa_status dsa_check_indices(const int32_t *idx, int B, int Lq, int start_pos,
+                             int k, int *bad_rows, void *stream);
+
 /* Self-test of failure detection (no counterpart in the pages): launches one
  * CTA that waits on a barrier nothing ever completes, gives up after
  * `limit_cycles` SM clock cycles (1 .. 2e9) and records the expiry in the

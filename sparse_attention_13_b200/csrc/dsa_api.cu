@@ -134,6 +134,28 @@ __global__ void selftest_wait_kernel(unsigned int* err, long long limit) {
   if (!done && threadIdx.x == 0) atomicOr(err, 1u);
 }
 
+// Checks that index rows have the canonical form dsa_indexer_topk writes
+// ([IDX] §1, §4: S_t is a subset of {s : 0 <= s < t} of size min(t, k)):
+// the first min(t, k) entries strictly ascending in [0, t), then -1.  One warp per row; each bad row adds 1 to *bad_rows.
+__global__ void check_indices_kernel(const int32_t* __restrict__ idx, int Lq, int start_pos, int k,
+                                     int* bad_rows) {
+  const size_t row = blockIdx.x;
+  const int t = start_pos + static_cast<int>(row % Lq);
+  const int n = min(t, k);
+  const int32_t* r = idx + row * k;
+  bool bad = false;
+  for (int e = threadIdx.x; e < k; e += 32) {
+    const int32_t v = r[e];
+    if (e < n) {
+      bad |= v < 0 || v >= t;
+      if (e > 0) bad |= v <= r[e - 1];
+    } else {
+      bad |= v != -1;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && threadIdx.x == 0) atomicAdd(bad_rows, 1);
+}
+
 }  // namespace dsa
 
 using namespace dsa;
@@ -259,6 +281,22 @@ dsa_status indexcache_forward(const char* pattern, int n_layers, const dsa_layer
                                     d.scale, L.out, L.lse, ws, ws_bytes, stream);
     if (st != DSA_OK) return st;
   }
+  return DSA_OK;
+}
+
+dsa_status dsa_check_indices(const int32_t* idx, int B, int Lq, int start_pos, int k, int* bad_rows,
+                             void* stream) {
+  if (!idx || !bad_rows) return set_error(DSA_ERR_INVALID_ARG, "dsa_check_indices: null pointer");
+  if (B < 1 || Lq < 1 || k < 1 || start_pos < 0)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_check_indices: sizes must be positive");
+  const long long rows = static_cast<long long>(B) * Lq;
+  if (rows > 2147483647ll) return set_error(DSA_ERR_UNSUPPORTED, "dsa_check_indices: too many rows");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(bad_rows, 0, sizeof(int), st);
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("dsa_check_indices: ") + cudaGetErrorString(e));
+  check_indices_kernel<<<static_cast<unsigned>(rows), 32, 0, st>>>(idx, Lq, start_pos, k, bad_rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("dsa_check_indices launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }
 

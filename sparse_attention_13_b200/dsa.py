@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_BAD_PATTERN",
 EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
            "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
-           "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout"]
+           "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout", "dsa_check_indices"]
 
 
 class DSAError(RuntimeError):
@@ -78,6 +78,8 @@ def lib():
         L.dsa_check_device_errors.restype = I
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
         L.dsa_selftest_wait_timeout.restype = I
+        L.dsa_check_indices.argtypes = [P, I, I, I, I, P, P]
+        L.dsa_check_indices.restype = I
         _lib = L
     return _lib
 
@@ -218,6 +220,18 @@ def indexer_launch_count() -> int:
 
 def check_device_errors(stream=None) -> None:
     _check(lib().dsa_check_device_errors(stream if stream is not None else _stream()))
+
+
+def check_indices(idx, start_pos: int = 0) -> int:
+    """Number of rows of idx [B, Lq, k] (int32, CUDA) that are not in the
+    canonical form dsa_indexer_topk writes (ascending positions below t, then
+    -1).  Synchronises the current stream."""
+    import torch
+    _need(idx, torch.int32, name="idx")
+    B, Lq, k = idx.shape
+    bad = torch.empty(1, dtype=torch.int32, device=idx.device)
+    _check(lib().dsa_check_indices(_ptr(idx), B, Lq, start_pos, k, _ptr(bad), _stream(idx)))
+    return int(bad.item())
 
 
 def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

@@ -118,3 +118,12 @@ def test_selftest_limit_validated_on_host(limit):
     # the failure-detection self-test refuses out-of-range limits before any
     # CUDA call
     assert dsa.lib().dsa_selftest_wait_timeout(limit, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_check_indices_validated_on_host():
+    lib = dsa.lib()
+    assert lib.dsa_check_indices(None, 1, 1, 0, 4, None, None) == dsa.DSA_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(16)  # never dereferenced: the sizes are refused first
+    assert lib.dsa_check_indices(fake, 0, 1, 0, 4, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_check_indices(fake, 1, 1, -1, 4, fake, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_check_indices(fake, 1, 1, 0, 0, fake, None) == dsa.DSA_ERR_INVALID_ARG

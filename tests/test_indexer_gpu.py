@@ -236,3 +236,21 @@ def test_decode_rows_at_the_slice_limit(dsa, oracle_mod, T):
     k_host = synth.tensor(seed, synth.K_IDX, synth.INT9, layer, (B, T, d))
     I = oracle_mod.indexer_row(q_host[0, 0], k_host[0], w_host[0, 0], T)
     check_topk_row(out[0, 0].cpu().numpy(), oracle_mod.topk_row(I, T, kk), I, kk)
+
+
+def test_check_indices_accepts_output_and_counts_planted_rows(dsa):
+    import torch
+    B, L, H, d, kk = 2, 3000, 64, 128, 512
+    q, k, w = indexer_inputs_host(37, B, L, L, H, d, integer=False)
+    idx = dsa.indexer_topk(to_dev_bf16(q), to_dev_bf16(k), to_dev_f32(w), kk)
+    assert dsa.check_indices(idx) == 0
+    bad = idx.clone()
+    bad[0, 5, 0] = 5            # position t itself is not visible
+    bad[0, 2000, 10] = bad[0, 2000, 9]   # not strictly ascending
+    bad[1, 100, 200] = 7        # padding must be -1 after min(t, k) entries
+    bad[1, 2999, kk - 1] = -1   # a full row must hold k positions
+    assert dsa.check_indices(bad) == 4
+    dec = dsa.indexer_topk(to_dev_bf16(q[:, :1]), to_dev_bf16(k), to_dev_f32(w[:, :1]), kk,
+                           start_pos=L)
+    assert dsa.check_indices(dec, start_pos=L) == 0
+    assert dsa.check_indices(torch.full_like(dec, -1), start_pos=L) == B

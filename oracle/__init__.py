@@ -48,6 +48,8 @@ def _load():
         lib.oracle_dense_attn_row.restype = None
         lib.oracle_masked_attn_row.argtypes = [P, P, i64, P, i64, P, i32, i32, i32, i32, i32, i32, f64, P, P]
         lib.oracle_masked_attn_row.restype = None
+        lib.oracle_dense_probs_row.argtypes = [P, P, i64, i32, i32, i32, f64, P]
+        lib.oracle_dense_probs_row.restype = None
         lib.oracle_indexcache_forward.argtypes = [
             ctypes.c_char_p, i32, P, P, P, P, P, i64, P, i64, i32, i32, i32, i32,
             i32, i32, i32, i32, i32, i32, f64, P, P, P, P]
@@ -136,6 +138,59 @@ def masked_attn_row(q_row, K, V, idx, T: int, scale: float, Dv: int | None = Non
                                    _p(idx), idx.shape[0], T, K.shape[0], n_h, Dqk, Dv,
                                    scale, _p(out), _p(lse))
     return out, lse
+
+
+def dense_probs_row(q_row, K, T: int, scale: float) -> np.ndarray:
+    """[IDX] §8.1: the dense attention weights alpha^dense_{t,s} of one query
+    row over P_t = {0 <= s < T}, per head.  q_row [n_h, Dqk] and K [>=T, Dqk]
+    (or a strided [rows, >=Dqk] view of the latent cache) as bf16 bits.
+    Returns [n_h, T] float64."""
+    q_row, K = _bits(q_row), _bits(K)
+    n_h, Dqk = q_row.shape
+    assert K.ndim == 2 and K.shape[1] >= Dqk and K.shape[0] >= T
+    alpha = np.zeros((n_h, T), dtype=np.float64)
+    _load().oracle_dense_probs_row(_p(q_row), _p(K), K.shape[1], T, n_h, Dqk,
+                                   float(scale), _p(alpha))
+    return alpha
+
+
+def captured_mass_row(alpha, idx) -> np.ndarray:
+    """[IDX] §8.1: CapturedMass@k = the dense weight that the selected set
+    holds, sum over s in S_t of alpha^dense_{t,s}, for each head (alpha
+    [n_h, T] from dense_probs_row; idx one index row, -1 entries skipped).
+    MissedMass@k is 1 minus it.  A query that sees nothing (T = 0) has S_t =
+    P_t = {} and is given mass 1: nothing of the dense weight is missed."""
+    alpha = np.asarray(alpha, dtype=np.float64)
+    sel = sorted({int(s) for s in np.asarray(idx) if s >= 0})
+    if alpha.shape[1] == 0:
+        assert not sel
+        return np.ones(alpha.shape[0])
+    assert all(s < alpha.shape[1] for s in sel)
+    return alpha[:, sel].sum(axis=1) if sel else np.zeros(alpha.shape[0])
+
+
+def overlap_row(a, b) -> int:
+    """|A intersect B| for two index rows (-1 entries skipped): the numerator
+    of [IDX] §8.4's adjacent-layer overlap |S^(l) & S^(l+1)| / k_idx and of
+    [IDX] §8.2's Recall@k."""
+    return len({int(s) for s in np.asarray(a) if s >= 0} & {int(s) for s in np.asarray(b) if s >= 0})
+
+
+def recall_row(s_oracle, s_model) -> float:
+    """[IDX] §8.2: Recall@k = |S^oracle & S^model| / |S^oracle|.  An empty
+    oracle set (T = 0) is given recall 1: there is nothing to miss."""
+    n = sum(1 for s in np.asarray(s_oracle) if s >= 0)
+    return 1.0 if n == 0 else overlap_row(s_oracle, s_model) / n
+
+
+def oracle_selection_row(alpha, T: int, k: int) -> np.ndarray:
+    """[IDX] §8.2: S_t^oracle = TopK_k { alpha^dense_{t,s} : s < t }.  The
+    page's alpha carries no head index; with n_h heads sharing one selection
+    the weights are averaged over heads (sum over h, divided by n_h) before
+    the top-k.  Same tie rule and row form as topk_row."""
+    alpha = np.asarray(alpha, dtype=np.float64)
+    mean = alpha.sum(axis=0) / alpha.shape[0] if T > 0 else np.zeros(0)
+    return topk_row(mean, T, k)
 
 
 def _ptr_array(arrs):

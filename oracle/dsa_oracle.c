@@ -159,6 +159,31 @@ void oracle_dense_attn_row(const uint16_t *q_row, const uint16_t *K, int64_t ks,
     free(pos);
 }
 
+/* Dense attention weights, one query row: [IDX] §8.1 (Captured Attention
+ * Mass), the dense weights alpha^dense_{t,s} that the selected set is scored
+ * against.  For each head h: e_s = scale * q[h] . K[s] for s in P_t =
+ * {0 <= s < T}; alpha[h][s] = exp(e_s - max e) / sum_s' exp(e_s' - max e).
+ * Written on its own (not through attend_list) so that its weights and the
+ * list form's log-sum-exp are two independent routes.
+ *   alpha : [n_h][T] double (written; nothing for T = 0) */
+void oracle_dense_probs_row(const uint16_t *q_row, const uint16_t *K, int64_t ks,
+                            int T, int n_h, int Dqk, double scale, double *alpha) {
+    for (int h = 0; h < n_h; ++h) {
+        double *a = alpha + (size_t)h * (size_t)T;
+        double m = -INFINITY;
+        for (int s = 0; s < T; ++s) {
+            double dot = 0.0;
+            for (int c = 0; c < Dqk; ++c)
+                dot += bf(q_row[(size_t)h * Dqk + c]) * bf(K[(int64_t)s * ks + c]);
+            a[s] = scale * dot;
+            if (a[s] > m) m = a[s];
+        }
+        double z = 0.0;
+        for (int s = 0; s < T; ++s) { a[s] = exp(a[s] - m); z += a[s]; }
+        for (int s = 0; s < T; ++s) a[s] /= z;
+    }
+}
+
 /* Index-mask formulation, one query row: [IDX] §6.4 (Transformers GLM
  * indexer).  Every position starts at mask -inf, the selected positions are
  * scattered to 0, the causal mask (-inf for s >= t) is added, and a dense

@@ -359,3 +359,94 @@ def test_decode_rows_use_start_pos(oracle_mod):
     assert idx[0, 0, 0].tolist() == list(range(Lk)) + [-1] * (64 - Lk)
     o, _ = oracle_mod.dense_attn_row(q[0, 0], kv[0], kv[0], Lk, 0.3)
     np.testing.assert_allclose(out[0, 0, 0], o, rtol=1e-13, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# selection quality: dense weights, CapturedMass, Recall, cross-layer overlap
+
+
+def test_dense_probs_two_keys_are_logistic(oracle_mod):
+    # Two keys: alpha_1 = 1 / (1 + exp(-(e_1 - e_0))), a closed form.
+    q = bf16([[1, 2], [-0.5, 1]])
+    K = bf16([[3, -1], [0.25, 2]])
+    scale = 0.7
+    alpha = oracle_mod.dense_probs_row(q, K, 2, scale)
+    qf, Kf = f32(q), f32(K)
+    for h in range(2):
+        d = scale * (qf[h] @ Kf[1] - qf[h] @ Kf[0])
+        np.testing.assert_allclose(alpha[h, 1], 1.0 / (1.0 + math.exp(-d)), rtol=1e-14)
+        np.testing.assert_allclose(alpha[h, 0], 1.0 / (1.0 + math.exp(d)), rtol=1e-14)
+
+
+def test_dense_probs_match_torch_softmax(oracle_mod):
+    T, n_h, D = 37, 3, 16
+    q, K, _ = _attn_inputs(8, T + 5, n_h, D)
+    alpha = oracle_mod.dense_probs_row(q, K, T, 0.4)
+    ref = torch.softmax(0.4 * torch.tensor(f32(q)) @ torch.tensor(f32(K)[:T]).T, dim=-1)
+    np.testing.assert_allclose(alpha, ref.numpy(), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(alpha.sum(axis=1), 1.0, rtol=1e-14)
+    # a zero query weighs every visible key alike
+    flat = oracle_mod.dense_probs_row(np.zeros_like(q), K, T, 0.4)
+    np.testing.assert_allclose(flat, 1.0 / T, rtol=1e-14)
+    assert oracle_mod.dense_probs_row(q, K, 0, 0.4).shape == (n_h, 0)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_captured_mass_equals_lse_ratio(oracle_mod, seed):
+    # sum_{s in S} alpha_s = exp(lse_S - lse_{P_t}): the weights of one C
+    # routine against the log-sum-exps of the attention routines.
+    rng = np.random.default_rng(seed)
+    T, k = 60, 16
+    q, K, V = _attn_inputs(seed + 20, T + 3, 4, 16, 8)
+    alpha = oracle_mod.dense_probs_row(q, K, T, 0.35)
+    idx = oracle_mod.topk_row(rng.normal(size=T), T, k)
+    mass = oracle_mod.captured_mass_row(alpha, idx)
+    _, l_sel = oracle_mod.sparse_attn_row(q, K, V, idx, 0.35)
+    _, l_all = oracle_mod.dense_attn_row(q, K, V, T, 0.35)
+    np.testing.assert_allclose(mass, np.exp(l_sel - l_all), rtol=1e-12)
+    assert np.all((mass > 0) & (mass < 1))
+
+
+def test_captured_mass_full_empty_and_additive(oracle_mod):
+    T, k = 25, 32
+    q, K, _ = _attn_inputs(3, T, 2, 8)
+    alpha = oracle_mod.dense_probs_row(q, K, T, 0.5)
+    full = oracle_mod.topk_row(np.zeros(T), T, k)          # all of P_t
+    np.testing.assert_allclose(oracle_mod.captured_mass_row(alpha, full), 1.0, rtol=1e-14)
+    np.testing.assert_array_equal(oracle_mod.captured_mass_row(alpha, -np.ones(k, np.int32)), 0.0)
+    a = np.array([0, 3, 7, -1], np.int32)
+    b = np.array([1, 2, 20, 24], np.int32)
+    ab = np.array([0, 1, 2, 3, 7, 20, 24, -1], np.int32)
+    np.testing.assert_allclose(oracle_mod.captured_mass_row(alpha, a)
+                               + oracle_mod.captured_mass_row(alpha, b),
+                               oracle_mod.captured_mass_row(alpha, ab), rtol=1e-14)
+    # T = 0: nothing visible, nothing missed
+    np.testing.assert_array_equal(
+        oracle_mod.captured_mass_row(np.zeros((2, 0)), -np.ones(4, np.int32)), 1.0)
+
+
+def test_overlap_and_recall_hand_example(oracle_mod):
+    a = np.array([1, 3, 5, -1], np.int32)
+    b = np.array([3, 4, 5, 6], np.int32)
+    assert oracle_mod.overlap_row(a, b) == 2
+    assert oracle_mod.overlap_row(b, b) == 4
+    assert oracle_mod.overlap_row(a, np.array([0, 2, 4, 6], np.int32)) == 0
+    assert oracle_mod.recall_row(a, b) == pytest.approx(2 / 3)
+    assert oracle_mod.recall_row(b, a) == pytest.approx(2 / 4)
+    assert oracle_mod.recall_row(-np.ones(4, np.int32), b) == 1.0
+
+
+def test_oracle_selection_is_topk_of_head_mean(oracle_mod):
+    # brute force on a tiny row: sort by (mean weight desc, s asc), keep k
+    T, k = 19, 6
+    q, K, _ = _attn_inputs(12, T, 3, 8)
+    alpha = oracle_mod.dense_probs_row(q, K, T, 0.6)
+    mean = alpha.mean(axis=0)
+    want = sorted(sorted(range(T), key=lambda s: (-mean[s], s))[:k])
+    assert oracle_mod.oracle_selection_row(alpha, T, k).tolist() == want
+    # one head: the head's own weights decide
+    a1 = oracle_mod.dense_probs_row(q[:1], K, T, 0.6)
+    want1 = sorted(sorted(range(T), key=lambda s: (-a1[0, s], s))[:k])
+    assert oracle_mod.oracle_selection_row(a1, T, k).tolist() == want1
+    # t < k: every visible position, then -1
+    assert oracle_mod.oracle_selection_row(alpha[:, :4], 4, k).tolist() == [0, 1, 2, 3, -1, -1]

@@ -695,6 +695,87 @@ def kernel_case(name, seq, reps):
     print(f"{name} seq={seq}: {e0.elapsed_time(e1) / reps:.3f} ms/launch", flush=True)
 
 
+def selection_quality(seq, layers=4, kk=2048):
+    """The selection-quality tools of [IDX] §8 on a short correlated synthetic
+    stack (B = 1, L = seq, `layers` layers, k = kk): per layer, the indexer's
+    own selection S^(l), the oracle selection TopK over the head-averaged
+    dense weights, CapturedMass@k and Recall@k of S^(l) and of the reused
+    S^(0), and the adjacent-layer overlap |S^(l-1) & S^(l)| / k, both with
+    the head weights redrawn per layer (the input recipe) and held at layer
+    0's.  Prints one
+    JSON line with the means (over rows t >= k, where selection matters) and
+    each tool kernel's CUDA-event time."""
+    import torch
+
+    from sparse_attention_13_b200 import dsa, synth
+    dev = torch.device("cuda", 0)
+    bf = torch.bfloat16
+    L, H, dI, n_h, Dqk = seq, 64, 128, 128, 576
+    scale = 1 / math.sqrt(Dqk)
+    times = {"dense_weights": 0.0, "topk_rows": 0.0, "index_overlap": 0.0, "captured_mass": 0.0}
+
+    def timed(name, fn):
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        r = fn()
+        e1.record()
+        e1.synchronize()
+        times[name] += e0.elapsed_time(e1)
+        return r
+
+    rows = slice(kk, L)               # rows whose selection is a real choice
+    n_sel = float(kk)
+    res = []
+    prev = first = prev_held = w0 = None
+    ws = torch.empty(dsa.indexer_topk_workspace(1, L, L, 0, H, dI, kk), dtype=torch.uint8, device=dev)
+    for l in range(layers):
+        qi = torch.empty((1, L, H, dI), dtype=bf, device=dev)
+        ki = torch.empty((1, L, dI), dtype=bf, device=dev)
+        w = torch.empty((1, L, H), dtype=torch.float32, device=dev)
+        q = torch.empty((1, L, n_h, Dqk), dtype=bf, device=dev)
+        kv = torch.empty((1, L, Dqk), dtype=bf, device=dev)
+        synth.fill_cuda(qi, SEED, synth.Q_IDX, synth.INT9, l, corr=True)
+        synth.fill_cuda(ki, SEED, synth.K_IDX, synth.INT9, l, corr=True)
+        synth.fill_cuda(w, SEED, synth.W, synth.POW2W, l)
+        synth.fill_cuda(q, SEED, synth.Q, synth.NORMAL, l, sigma=0.5, corr=True)
+        synth.fill_cuda(kv, SEED, synth.KV, synth.NORMAL, l, sigma=0.5, corr=True)
+        own = dsa.indexer_topk(qi, ki, w, kk, ws=ws)
+        first = own if first is None else first
+        lse_d, mw = timed("dense_weights", lambda: dsa.dense_weights(q, kv, scale=scale))
+        s_or = timed("topk_rows", lambda: dsa.topk_rows(mw, kk))
+        entry = {"layer": l}
+        for tag, sel in (("own", own), ("reused", first)):
+            lse_s = torch.empty_like(lse_d)
+            dsa.sparse_attn(q, kv, kv, sel, scale, D_v=512, lse=lse_s)
+            mass = timed("captured_mass", lambda: dsa.captured_mass(lse_s, lse_d))
+            inter = timed("index_overlap", lambda: dsa.index_overlap(s_or, sel))
+            entry[f"captured_mass_{tag}"] = float(mass[0, rows].mean())
+            entry[f"recall_{tag}"] = float(inter[0, rows].float().mean()) / n_sel
+        if prev is not None:
+            inter = timed("index_overlap", lambda: dsa.index_overlap(prev, own))
+            entry["overlap_prev"] = float(inter[0, rows].float().mean()) / n_sel
+        # the same layer with layer 0's head weights: the overlap then follows
+        # the 0.9 correlation of q_idx and k_idx alone
+        held = own if l == 0 else dsa.indexer_topk(qi, ki, w0, kk, ws=ws)
+        if prev_held is not None:
+            inter = timed("index_overlap", lambda: dsa.index_overlap(prev_held, held))
+            entry["overlap_prev_w_held"] = float(inter[0, rows].float().mean()) / n_sel
+        prev, prev_held = own, held
+        w0 = w if l == 0 else w0
+        res.append(entry)
+    dsa.check_device_errors()
+    flops = 2 * 2 * n_h * Dqk * (L * (L - 1) // 2)   # two passes of logits per dense call
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12          # FMA units x 2 flop x max clock
+    dw_ms = times["dense_weights"] / layers
+    print(json.dumps({
+        "tool": "selection_quality", "workload": f"B=1, L={L}, {layers} correlated layers, k={kk}, "
+        "indexer H_I=64 d_I=128, MLA 128 heads 576/512", "data": "synthetic",
+        "per_layer": res, "ms_per_layer": {k: v / layers for k, v in times.items()},
+        "dense_weights_roofline": {"bound": "alu", "achieved": flops / dw_ms / 1e9, "unit": "TFLOP/s",
+                                   "peak": fp32_peak, "frac": flops / dw_ms / 1e9 / fp32_peak,
+                                   "peak_kind": "fp32 FMA issue at 1965 MHz (derived)"}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -704,9 +785,13 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="override the prefill length (testing)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default="",
-                    help="profiling: indexer|attn|decode_idx|decode_attn|decode_step")
+                    help="profiling: indexer|attn|decode_idx|decode_attn|decode_step; "
+                         "quality runs the selection-quality tools")
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
+    if args.kernel_case == "quality":
+        selection_quality(args.seq or 8192)
+        return
     if args.kernel_case:
         kernel_case(args.kernel_case, args.seq or 16384, args.reps)
         return

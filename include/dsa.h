@@ -176,6 +176,51 @@ long long dsa_indexer_launch_count(void);
 dsa_status dsa_check_indices(const int32_t *idx, int B, int Lq, int start_pos,
                              int k, int *bad_rows, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Selection quality ([IDX] §8, how index quality is judged).  Tools for short
+ * contexts; they are not on the layer loop's path and run on CUDA cores.
+ *
+ * dsa_dense_weights: dense causal attention statistics of each query row
+ * (row i at t = start_pos + i sees s < t; q, kbuf, k_row_stride as in
+ * dsa_sparse_attn):
+ *   lse_dense [B, Lq, n_h] f32 (written): log sum_{s<t} exp(scale q[t,h].K[s])
+ *     (natural log; -inf for t = 0);
+ *   mean_w [B, Lq, Lk] f32 (written for s < t only; may be NULL): the dense
+ *     weights alpha^dense_{t,s} of §8.1 averaged over heads,
+ *     (1/n_h) sum_h exp(scale q[t,h].K[s] - lse_dense[t,h]).
+ * Supported: n_h <= 128, D_qk <= 576 and a multiple of 8, k_row_stride a
+ * multiple of 8.  Work is O(sum_t t * n_h * D_qk) per pass, two passes. */
+dsa_status dsa_dense_weights(const dsa_bf16 *q, const dsa_bf16 *kbuf,
+                             int64_t k_row_stride, int B, int Lq, int Lk,
+                             int start_pos, int n_h, int D_qk, float scale,
+                             float *lse_dense, float *mean_w, void *stream);
+
+/* dsa_topk_rows: TopK_k over dense score rows, the oracle selection of §8.2
+ * (S^oracle = TopK_k of alpha^dense over s < t) when given mean_w.  Row
+ * (b, i) is scores + (b*Lq + i)*row_stride and holds t = start_pos + i
+ * finite scores; requires start_pos + Lq - 1 <= row_stride.  Output
+ * idx [B, Lq, k] int32 in the row form of dsa_indexer_topk: ties go to the
+ * lower position, positions ascending, then -1. */
+dsa_status dsa_topk_rows(const float *scores, int64_t row_stride, int B, int Lq,
+                         int start_pos, int k, int32_t *idx, void *stream);
+
+/* dsa_index_overlap: inter[r] = |A_r & B_r| for `rows` pairs of index rows
+ * of length k in the row form above (ascending, then -1; rows that are not
+ * give an unspecified count but no out-of-range read).  inter / k is the
+ * adjacent-layer overlap of §8.4 for A = S^(l), B = S^(l+1); inter /
+ * |S^oracle| is Recall@k of §8.2 for A = S^oracle, B = S^model. */
+dsa_status dsa_index_overlap(const int32_t *a, const int32_t *b, int64_t rows,
+                             int k, int32_t *inter, void *stream);
+
+/* dsa_captured_mass: CapturedMass@k of §8.1 per (row, head):
+ * mass[e] = exp(lse_sel[e] - lse_dense[e]), which equals the dense weight
+ * sum over the selected set when lse_sel comes from dsa_sparse_attn on that
+ * set and lse_dense from dsa_dense_weights with the same q, K and scale.  A
+ * row that sees nothing (lse_dense = -inf) gets mass 1.  MissedMass@k is
+ * 1 - mass.  n elements, all f32 device arrays. */
+dsa_status dsa_captured_mass(const float *lse_sel, const float *lse_dense,
+                             int64_t n, float *mass, void *stream);
+
 /* Self-test of failure detection (no counterpart in the pages): launches one
  * CTA that waits on a barrier nothing ever completes, gives up after
  * `limit_cycles` SM clock cycles (1 .. 2e9) and records the expiry in the

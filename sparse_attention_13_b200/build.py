@@ -18,7 +18,8 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-s
                 "-cudart", "static", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 LIBS = {
-    "libdsa.so": ["dsa_api.cu", "indexer_topk.cu", "decode_indexer.cu", "sparse_attn.cu", "noalloc.cu"],
+    "libdsa.so": ["dsa_api.cu", "indexer_topk.cu", "decode_indexer.cu", "sparse_attn.cu", "noalloc.cu",
+                  "selection_quality.cu"],
     "libdsa_synth.so": ["synth.cu"],
 }
 DEPS = ["dsa_ptx.cuh", "dsa_internal.h"]

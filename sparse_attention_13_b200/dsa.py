@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_BAD_PATTERN",
 EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
            "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
-           "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout", "dsa_check_indices"]
+           "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout", "dsa_check_indices",
+           "dsa_dense_weights", "dsa_topk_rows", "dsa_index_overlap", "dsa_captured_mass"]
 
 
 class DSAError(RuntimeError):
@@ -80,6 +81,15 @@ def lib():
         L.dsa_selftest_wait_timeout.restype = I
         L.dsa_check_indices.argtypes = [P, I, I, I, I, P, P]
         L.dsa_check_indices.restype = I
+        F32 = ctypes.c_float
+        L.dsa_dense_weights.argtypes = [P, P, I64, I, I, I, I, I, I, F32, P, P, P]
+        L.dsa_dense_weights.restype = I
+        L.dsa_topk_rows.argtypes = [P, I64, I, I, I, I, P, P]
+        L.dsa_topk_rows.restype = I
+        L.dsa_index_overlap.argtypes = [P, P, I64, I, P, P]
+        L.dsa_index_overlap.restype = I
+        L.dsa_captured_mass.argtypes = [P, P, I64, P, P]
+        L.dsa_captured_mass.restype = I
         _lib = L
     return _lib
 
@@ -232,6 +242,64 @@ def check_indices(idx, start_pos: int = 0) -> int:
     bad = torch.empty(1, dtype=torch.int32, device=idx.device)
     _check(lib().dsa_check_indices(_ptr(idx), B, Lq, start_pos, k, _ptr(bad), _stream(idx)))
     return int(bad.item())
+
+
+def dense_weights(q, kv, *, Lk: int | None = None, start_pos: int = 0, scale: float,
+                  D_qk: int | None = None, mean_weights: bool = True):
+    """Dense causal attention statistics ([IDX] §8.1) of q [B, Lq, n_h, D_qk]
+    against the rows of kv [B, Lk, row] (bf16, CUDA; the first D_qk columns
+    are the keys).  Returns (lse_dense [B, Lq, n_h] f32, mean_w [B, Lq, Lk]
+    f32 or None); mean_w holds the head-averaged dense weights for s < t and
+    zeros elsewhere."""
+    import torch
+    _need(q, torch.bfloat16, name="q")
+    _need(kv, torch.bfloat16, name="kv")
+    B, Lq, n_h, Dq = q.shape
+    D_qk = Dq if D_qk is None else D_qk
+    assert D_qk == Dq, "q's last dimension is D_qk"
+    Lk = kv.shape[1] if Lk is None else Lk
+    lse = torch.empty((B, Lq, n_h), dtype=torch.float32, device=q.device)
+    mw = torch.zeros((B, Lq, Lk), dtype=torch.float32, device=q.device) if mean_weights else None
+    _check(lib().dsa_dense_weights(_ptr(q), _ptr(kv), kv.shape[2], B, Lq, Lk, start_pos, n_h, D_qk,
+                                   float(scale), _ptr(lse), _ptr(mw), _stream(q)))
+    return lse, mw
+
+
+def topk_rows(scores, k: int, start_pos: int = 0):
+    """TopK_k over dense score rows scores [B, Lq, W] (f32, CUDA); row i holds
+    start_pos + i scores.  The oracle selection of [IDX] §8.2 when given the
+    head-averaged dense weights.  Returns idx [B, Lq, k] int32."""
+    import torch
+    _need(scores, torch.float32, name="scores")
+    B, Lq, W = scores.shape
+    idx = torch.empty((B, Lq, k), dtype=torch.int32, device=scores.device)
+    _check(lib().dsa_topk_rows(_ptr(scores), W, B, Lq, start_pos, k, _ptr(idx), _stream(scores)))
+    return idx
+
+
+def index_overlap(a, b):
+    """|A & B| per row of two index tensors [..., k] (int32, CUDA, row form
+    of indexer_topk).  Returns int32 counts of shape a.shape[:-1]."""
+    import torch
+    _need(a, torch.int32, name="a")
+    _need(b, torch.int32, shape=a.shape, name="b")
+    k = a.shape[-1]
+    rows = a.numel() // k
+    inter = torch.empty(a.shape[:-1], dtype=torch.int32, device=a.device)
+    _check(lib().dsa_index_overlap(_ptr(a), _ptr(b), rows, k, _ptr(inter), _stream(a)))
+    return inter
+
+
+def captured_mass(lse_sel, lse_dense):
+    """CapturedMass@k ([IDX] §8.1) = exp(lse_sel - lse_dense) elementwise (f32,
+    CUDA, same shape); 1 where the row sees nothing."""
+    import torch
+    _need(lse_sel, torch.float32, name="lse_sel")
+    _need(lse_dense, torch.float32, shape=lse_sel.shape, name="lse_dense")
+    mass = torch.empty_like(lse_sel)
+    _check(lib().dsa_captured_mass(_ptr(lse_sel), _ptr(lse_dense), lse_sel.numel(), _ptr(mass),
+                                   _stream(lse_sel)))
+    return mass
 
 
 def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

@@ -127,3 +127,21 @@ def test_check_indices_validated_on_host():
     assert lib.dsa_check_indices(fake, 0, 1, 0, 4, fake, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_check_indices(fake, 1, 1, -1, 4, fake, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_check_indices(fake, 1, 1, 0, 0, fake, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_selection_quality_tools_validated_on_host():
+    lib = dsa.lib()
+    fake = ctypes.c_void_p(16)  # never dereferenced: the arguments are refused first
+    E = dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_dense_weights(None, fake, 576, 1, 1, 1, 0, 128, 576, 1.0, fake, None, None) == E
+    assert lib.dsa_dense_weights(fake, fake, 576, 1, 3, 1, 0, 128, 576, 1.0, fake, None, None) == E
+    assert lib.dsa_dense_weights(fake, fake, 576, 1, 1, 1, 0, 129, 576, 1.0, fake, None,
+                                 None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_dense_weights(fake, fake, 576, 1, 1, 1, 0, 8, 100, 1.0, fake, None,
+                                 None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_dense_weights(fake, fake, 60, 1, 1, 1, 0, 8, 64, 1.0, fake, None, None) == E
+    assert lib.dsa_topk_rows(fake, 10, 1, 2, 10, 4, fake, None) == E     # t = 11 > row
+    assert lib.dsa_topk_rows(fake, 10, 1, 2, 0, 0, fake, None) == E
+    assert lib.dsa_index_overlap(fake, None, 4, 8, fake, None) == E
+    assert lib.dsa_index_overlap(fake, fake, 0, 8, fake, None) == E
+    assert lib.dsa_captured_mass(fake, fake, 0, fake, None) == E

@@ -193,6 +193,30 @@ def oracle_selection_row(alpha, T: int, k: int) -> np.ndarray:
     return topk_row(mean, T, k)
 
 
+def csa_visible(t: int, m: int) -> int:
+    """[IDX] §5.2 (CSA indexer over compressed blocks): compressed block s is
+    visible to query t iff s < floor(t / m), so query t sees floor(t / m)
+    blocks."""
+    assert t >= 0 and m >= 1
+    return t // m
+
+
+def csa_indexer_topk_row(q_row, k_cmp, w_row, t: int, m: int, k: int):
+    """[IDX] §5.2: I[t,s] = sum_j w[t,j] ReLU(q[t,j] . K^IComp[s]) over the
+    visible compressed blocks s < floor(t/m), then S_t^CSA = TopK_k.  Same
+    score, tie rule and row form as the token-level indexer.  Returns (I, idx)."""
+    T = csa_visible(t, m)
+    I = indexer_row(q_row, k_cmp, w_row, T)
+    return I, topk_row(I, T, k)
+
+
+def csa_attn_row(q_row, c_cmp, idx, scale: float, Dv: int | None = None):
+    """[IDX] §5.2: o_t = CoreAttn(q_t, {C_s^Comp : s in S_t^CSA}) with keys and
+    values from the same compressed entries (shared-KV MQA; for the MLA shape
+    V is the first Dv columns).  Returns (out, lse)."""
+    return sparse_attn_row(q_row, c_cmp, c_cmp, idx, scale, Dv)
+
+
 def _ptr_array(arrs):
     arr = (ctypes.c_void_p * len(arrs))()
     for i, a in enumerate(arrs):

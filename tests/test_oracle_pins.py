@@ -450,3 +450,48 @@ def test_oracle_selection_is_topk_of_head_mean(oracle_mod):
     assert oracle_mod.oracle_selection_row(a1, T, k).tolist() == want1
     # t < k: every visible position, then -1
     assert oracle_mod.oracle_selection_row(alpha[:, :4], 4, k).tolist() == [0, 1, 2, 3, -1, -1]
+
+
+# --------------------------------------------------------------------------
+# CSA indexer over compressed blocks: s < floor(t / m)
+
+
+def test_csa_visibility_follows_floor_rule(oracle_mod):
+    # one head, w = 1, block s scores s + 1: the top-2 of the visible blocks
+    # are the last two below floor(t / 4)
+    m, nb, d = 4, 8, 8
+    q = bf16(np.eye(1, d))
+    kc = bf16(np.arange(1, nb + 1)[:, None] * np.eye(1, d))
+    w = np.ones(1, np.float32)
+    for t in range(0, m * nb + 1):
+        T = t // m
+        assert oracle_mod.csa_visible(t, m) == T
+        I, idx = oracle_mod.csa_indexer_topk_row(q, kc, w, t, m, 2)
+        np.testing.assert_array_equal(I, np.arange(1, T + 1))
+        want = [s for s in (T - 2, T - 1) if s >= 0]
+        assert idx.tolist() == want + [-1] * (2 - len(want))
+    # t = 7 sees block 0 only; t = 8 also block 1
+    assert oracle_mod.csa_indexer_topk_row(q, kc, w, 7, m, 4)[1].tolist() == [0, -1, -1, -1]
+    assert oracle_mod.csa_indexer_topk_row(q, kc, w, 8, m, 4)[1].tolist() == [0, 1, -1, -1]
+
+
+def test_csa_with_m_1_is_the_token_indexer(oracle_mod):
+    rng = np.random.default_rng(4)
+    H, d, L, k = 4, 16, 40, 7
+    q = bf16(rng.normal(size=(H, d)))
+    kk = bf16(rng.normal(size=(L, d)))
+    w = rng.normal(size=H).astype(np.float32)
+    for t in (0, 1, 6, 7, 8, 39):
+        I, idx = oracle_mod.csa_indexer_topk_row(q, kk, w, t, 1, k)
+        I2 = oracle_mod.indexer_row(q, kk, w, t)
+        np.testing.assert_array_equal(I, I2)
+        np.testing.assert_array_equal(idx, oracle_mod.topk_row(I2, t, k))
+
+
+def test_csa_attention_reads_selected_compressed_entries(oracle_mod):
+    # keys and values both come from the selected compressed entries: with a
+    # single selected entry the output is that entry's value columns
+    q, C, _ = _attn_inputs(9, 6, 2, 16)
+    out, lse = oracle_mod.csa_attn_row(q, C, np.array([3, -1, -1], np.int32), 0.5, Dv=8)
+    np.testing.assert_allclose(out, np.broadcast_to(f32(C)[3, :8], out.shape), rtol=1e-15)
+    np.testing.assert_allclose(lse, 0.5 * f32(q) @ f32(C)[3], rtol=1e-14)

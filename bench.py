@@ -695,6 +695,65 @@ def kernel_case(name, seq, reps):
     print(f"{name} seq={seq}: {e0.elapsed_time(e1) / reps:.3f} ms/launch", flush=True)
 
 
+def csa_layer(seq, kk=512, m=4, reps=2):
+    """One CSA-style layer ([IDX] §5.2, the V4 settings of §5.3: m = 4, 64
+    indexer heads x 128, k = 512) at B = 1, L = seq: the indexer over the
+    floor(t/m) visible compressed blocks with top-k, then MLA attention over
+    the selected compressed entries.  Synthetic compressed keys and latent
+    entries (the gated compression needs weights).  Prints one JSON line with
+    CUDA-event times per call and the tensor-pipe roofline of each."""
+    import torch
+
+    from sparse_attention_13_b200 import dsa, synth
+    dev = torch.device("cuda", 0)
+    bf = torch.bfloat16
+    L, H, dI = seq, 64, 128
+    N = L // m
+    qi = torch.empty((1, L, H, dI), dtype=bf, device=dev)
+    kc = torch.empty((1, N, dI), dtype=bf, device=dev)
+    w = torch.empty((1, L, H), dtype=torch.float32, device=dev)
+    synth.fill_cuda(qi, SEED, synth.Q_IDX, synth.INT9, 0)
+    synth.fill_cuda(kc, SEED, synth.K_IDX, synth.INT9, 0)
+    synth.fill_cuda(w, SEED, synth.W, synth.POW2W, 0)
+    idx = torch.empty((1, L, kk), dtype=torch.int32, device=dev)
+    ws = torch.empty(dsa.csa_indexer_topk_workspace(1, L, N, 0, m, H, dI, kk), dtype=torch.uint8, device=dev)
+    q = torch.empty((1, L, 128, 576), dtype=bf, device=dev)
+    c = torch.empty((1, N, 576), dtype=bf, device=dev)
+    synth.fill_cuda(q, SEED, synth.Q, synth.NORMAL, 0, sigma=0.5)
+    synth.fill_cuda(c, SEED, synth.KV, synth.NORMAL, 0, sigma=0.5)
+    out = torch.empty((1, L, 128, 512), dtype=bf, device=dev)
+    aws = torch.empty(max(dsa.sparse_attn_workspace(1, L, 128, 512, kk), 16), dtype=torch.uint8, device=dev)
+    scale = 1 / math.sqrt(576)
+    run_idx = lambda: dsa.csa_indexer_topk(qi, kc, w, kk, m=m, out=idx, ws=ws)
+    run_attn = lambda: dsa.csa_sparse_attn(q, c, idx, scale, m=m, D_v=512, out=out, ws=aws)
+
+    def ms_of(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    t_idx, t_attn = ms_of(run_idx), ms_of(run_attn)
+    dsa.check_device_errors()
+    peak = measured_peaks()[1]
+    pairs = sum(t // m for t in range(L))
+    idx_flops = 2 * H * dI * pairs
+    attn_flops = 2 * 128 * (576 + 512) * sum(min(t // m, kk) for t in range(L))
+    print(json.dumps({
+        "tool": "csa_layer", "workload": f"B=1, L={L}, m={m}, N_cmp={N}, k={kk}, indexer H_I=64 d_I=128, "
+        "MLA 128 heads 576/512 over compressed entries", "data": "synthetic",
+        "indexer_ms": t_idx, "attn_ms": t_attn,
+        "indexer_roofline": {"bound": "tensor", "achieved": idx_flops / t_idx / 1e9, "unit": "TFLOP/s",
+                             "peak": peak, "frac": idx_flops / t_idx / 1e9 / peak},
+        "attn_roofline": {"bound": "tensor", "achieved": attn_flops / t_attn / 1e9, "unit": "TFLOP/s",
+                          "peak": peak, "frac": attn_flops / t_attn / 1e9 / peak}}), flush=True)
+
+
 def selection_quality(seq, layers=4, kk=2048):
     """The selection-quality tools of [IDX] §8 on a short correlated synthetic
     stack (B = 1, L = seq, `layers` layers, k = kk): per layer, the indexer's
@@ -786,11 +845,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default="",
                     help="profiling: indexer|attn|decode_idx|decode_attn|decode_step; "
-                         "quality runs the selection-quality tools")
+                         "quality runs the selection-quality tools, csa one CSA-style layer")
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
     if args.kernel_case == "quality":
         selection_quality(args.seq or 8192)
+        return
+    if args.kernel_case == "csa":
+        csa_layer(args.seq or 200000, reps=args.reps)
         return
     if args.kernel_case:
         kernel_case(args.kernel_case, args.seq or 16384, args.reps)

@@ -177,6 +177,44 @@ dsa_status dsa_check_indices(const int32_t *idx, int B, int Lq, int start_pos,
                              int k, int *bad_rows, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * CSA-style selection over compressed blocks ([IDX] §5.2).  Every m tokens'
+ * KV are compressed into one entry (the gated compression needs trained
+ * weights and is not computed here: the compressed indexer keys and latent
+ * entries are inputs).  Query row i at t = start_pos + i sees the compressed
+ * blocks s < floor(t/m):
+ *   I[t,s] = sum_j w[t,j] * ReLU(q_idx[t,j,:] . k_cmp[s,:]),
+ *   S_t^CSA = TopK_k { I[t,s] : s < floor(t/m) },
+ * with the tie rule and row form of dsa_indexer_topk, and the main attention
+ * reads the selected compressed entries as shared K and V.
+ *   q_idx [B, Lq, H_I, d_I] bf16; k_cmp [B, N_cmp, d_I] bf16; w [B, Lq, H_I]
+ *   f32; idx [B, Lq, k] int32 (written).
+ * Requires floor((start_pos + Lq - 1) / m) <= N_cmp, m >= 1, and the
+ * dsa_indexer_topk limits on H_I, d_I, k.  Several query rows (Lq > 1) with
+ * m > 1 need start_pos to be a multiple of m (chunked prefill on block
+ * boundaries), else DSA_ERR_UNSUPPORTED.  The rows are regrouped by t mod m
+ * into m sequences of one fused indexer launch, so the workspace holds a
+ * phase-major copy of q_idx, w and the keys besides the indexer's own. */
+size_t dsa_csa_indexer_topk_workspace(int B, int Lq, int N_cmp, int start_pos,
+                                      int m, int H_I, int d_I, int k);
+dsa_status dsa_csa_indexer_topk(const dsa_bf16 *q_idx, const dsa_bf16 *k_cmp,
+                                const float *w, int B, int Lq, int N_cmp,
+                                int start_pos, int m, int H_I, int d_I, int k,
+                                int32_t *idx, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/* Attention over the selected compressed entries ([IDX] §5.2, CoreAttn with
+ * keys and values from the same entries): dsa_sparse_attn over the rows
+ * c_cmp + (b*N_cmp + s)*row_stride, with the CSA visibility check above.
+ * Valid index entries must satisfy 0 <= s < floor(t/m).  Workspace:
+ * dsa_sparse_attn_workspace(B, Lq, n_h, D_v, k). */
+dsa_status dsa_csa_sparse_attn(const dsa_bf16 *q, const dsa_bf16 *c_cmp,
+                               int64_t row_stride, const int32_t *idx, int B,
+                               int Lq, int N_cmp, int start_pos, int m, int n_h,
+                               int D_qk, int D_v, int k, float scale,
+                               dsa_bf16 *out, float *lse, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Selection quality ([IDX] §8, how index quality is judged).  Tools for short
  * contexts; they are not on the layer loop's path and run on CUDA cores.
  *

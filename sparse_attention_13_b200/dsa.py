@@ -23,7 +23,8 @@ EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "dsa_sparse_attn_workspace", "dsa_sparse_attn", "indexcache_forward_workspace",
            "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
            "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout", "dsa_check_indices",
-           "dsa_dense_weights", "dsa_topk_rows", "dsa_index_overlap", "dsa_captured_mass"]
+           "dsa_dense_weights", "dsa_topk_rows", "dsa_index_overlap", "dsa_captured_mass",
+           "dsa_csa_indexer_topk_workspace", "dsa_csa_indexer_topk", "dsa_csa_sparse_attn"]
 
 
 class DSAError(RuntimeError):
@@ -90,6 +91,13 @@ def lib():
         L.dsa_index_overlap.restype = I
         L.dsa_captured_mass.argtypes = [P, P, I64, P, P]
         L.dsa_captured_mass.restype = I
+        L.dsa_csa_indexer_topk_workspace.argtypes = [I, I, I, I, I, I, I, I]
+        L.dsa_csa_indexer_topk_workspace.restype = SZ
+        L.dsa_csa_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, P, SZ, P]
+        L.dsa_csa_indexer_topk.restype = I
+        L.dsa_csa_sparse_attn.argtypes = [P, P, I64, P, I, I, I, I, I, I, I, I, I, F32, P, P, P,
+                                          SZ, P]
+        L.dsa_csa_sparse_attn.restype = I
         _lib = L
     return _lib
 
@@ -242,6 +250,58 @@ def check_indices(idx, start_pos: int = 0) -> int:
     bad = torch.empty(1, dtype=torch.int32, device=idx.device)
     _check(lib().dsa_check_indices(_ptr(idx), B, Lq, start_pos, k, _ptr(bad), _stream(idx)))
     return int(bad.item())
+
+
+def csa_indexer_topk_workspace(B, Lq, N_cmp, start_pos, m, H_I, d_I, k) -> int:
+    return int(lib().dsa_csa_indexer_topk_workspace(B, Lq, N_cmp, start_pos, m, H_I, d_I, k))
+
+
+def csa_indexer_topk(q_idx, k_cmp, w, k: int, *, m: int, start_pos: int = 0, out=None, ws=None):
+    """CSA-style indexer + top-k over compressed blocks ([IDX] §5.2): row i at
+    t = start_pos + i scores the blocks s < floor(t/m) of k_cmp [B, N_cmp,
+    d_I].  q_idx [B, Lq, H_I, d_I] bf16, w [B, Lq, H_I] f32.  Returns idx
+    [B, Lq, k] int32 (ascending block ids, then -1)."""
+    import torch
+    B, Lq, H, d = q_idx.shape
+    N = k_cmp.shape[1]
+    _need(q_idx, torch.bfloat16, name="q_idx")
+    _need(k_cmp, torch.bfloat16, (B, N, d), "k_cmp")
+    _need(w, torch.float32, (B, Lq, H), "w")
+    if out is None:
+        out = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device)
+    _need(out, torch.int32, (B, Lq, k), "out")
+    need = csa_indexer_topk_workspace(B, Lq, N, start_pos, m, H, d, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_idx.device)
+    _check(lib().dsa_csa_indexer_topk(_ptr(q_idx), _ptr(k_cmp), _ptr(w), B, Lq, N, start_pos, m, H, d,
+                                      k, _ptr(out), _ptr(ws), ws.numel(), _stream(q_idx)))
+    return out
+
+
+def csa_sparse_attn(q, c_cmp, idx, scale: float, *, m: int, D_v: int, start_pos: int = 0,
+                    out=None, lse=None, ws=None):
+    """Attention over the selected compressed entries ([IDX] §5.2): keys and
+    values are the rows of c_cmp [B, N_cmp, C] (K = the first D_qk columns,
+    V = the first D_v).  q [B, Lq, n_h, D_qk] bf16; idx from csa_indexer_topk."""
+    import torch
+    B, Lq, n_h, D_qk = q.shape
+    N = c_cmp.shape[1]
+    k = idx.shape[2]
+    _need(q, torch.bfloat16, name="q")
+    _need(c_cmp, torch.bfloat16, name="c_cmp")
+    _need(idx, torch.int32, (B, Lq, k), "idx")
+    if out is None:
+        out = torch.empty((B, Lq, n_h, D_v), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (B, Lq, n_h, D_v), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (B, Lq, n_h), "lse")
+    need = sparse_attn_workspace(B, Lq, n_h, D_v, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().dsa_csa_sparse_attn(_ptr(q), _ptr(c_cmp), c_cmp.shape[2], _ptr(idx), B, Lq, N,
+                                     start_pos, m, n_h, D_qk, D_v, k, float(scale), _ptr(out),
+                                     _ptr(lse), _ptr(ws), ws.numel(), _stream(q)))
+    return out
 
 
 def dense_weights(q, kv, *, Lk: int | None = None, start_pos: int = 0, scale: float,

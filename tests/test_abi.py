@@ -145,3 +145,27 @@ def test_selection_quality_tools_validated_on_host():
     assert lib.dsa_index_overlap(fake, None, 4, 8, fake, None) == E
     assert lib.dsa_index_overlap(fake, fake, 0, 8, fake, None) == E
     assert lib.dsa_captured_mass(fake, fake, 0, fake, None) == E
+
+
+def test_csa_entry_points_validated_on_host():
+    lib = dsa.lib()
+    fake = ctypes.c_void_p(16)  # never dereferenced: the arguments are refused first
+    E = dsa.DSA_ERR_INVALID_ARG
+    # (q, k_cmp, w, B, Lq, N_cmp, start_pos, m, H, d, k, idx, ws, ws_bytes, stream)
+    assert lib.dsa_csa_indexer_topk(None, fake, fake, 1, 8, 2, 0, 4, 64, 128, 8, fake, fake, 1 << 20, None) == E
+    assert lib.dsa_csa_indexer_topk(fake, fake, fake, 1, 8, 2, 0, 0, 64, 128, 8, fake, fake, 1 << 20, None) == E
+    # floor((0 + 12 - 1) / 4) = 2 > N_cmp = 1
+    assert lib.dsa_csa_indexer_topk(fake, fake, fake, 1, 12, 1, 0, 4, 64, 128, 8, fake, fake, 1 << 20, None) == E
+    # several rows from a start that is not on a block boundary
+    assert lib.dsa_csa_indexer_topk(fake, fake, fake, 1, 8, 10, 6, 4, 64, 128, 8, fake, fake, 1 << 20,
+                                    None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_csa_indexer_topk_workspace(1, 8, 10, 0, 0, 64, 128, 8) == 0
+    assert lib.dsa_csa_indexer_topk_workspace(2, 4096, 1024, 0, 4, 64, 128, 512) > \
+        2 * 4096 * 64 * 128 * 2  # holds the phase-major copy of q_idx
+    # (q, c, stride, idx, B, Lq, N, start, m, n_h, Dqk, Dv, k, scale, out, lse, ws, ws_bytes, stream)
+    assert lib.dsa_csa_sparse_attn(None, fake, 576, fake, 1, 8, 2, 0, 4, 128, 576, 512, 8, 1.0,
+                                   fake, None, fake, 0, None) == E
+    assert lib.dsa_csa_sparse_attn(fake, fake, 576, fake, 1, 12, 1, 0, 4, 128, 576, 512, 8, 1.0,
+                                   fake, None, fake, 0, None) == E
+    assert lib.dsa_csa_sparse_attn(fake, fake, 500, fake, 1, 8, 2, 0, 4, 128, 576, 512, 8, 1.0,
+                                   fake, None, fake, 0, None) == E

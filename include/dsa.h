@@ -215,7 +215,7 @@ dsa_status dsa_csa_sparse_attn(const dsa_bf16 *q, const dsa_bf16 *c_cmp,
                                size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
- * Selection quality ([IDX] §8, how index quality is judged).  Tools for short
+ * Selection quality ([IDX] §8, how index quality is evaluated).  Tools for short
  * contexts; they are not on the layer loop's path and run on CUDA cores.
  *
  * dsa_dense_weights: dense causal attention statistics of each query row

@@ -1,6 +1,6 @@
 // selection_quality.cu -- measurement tools for index selections, after
 // [IDX] "注意力机制中的 Index：从位置下标到预算检索" §8 (how index quality is
-// judged):
+// evaluated):
 //   - dense_weights_kernel: the dense attention weights alpha^dense_{t,s}
 //     that a selection is scored against (§8.1), averaged over heads, and the
 //     dense log-sum-exp per head;

@@ -68,6 +68,10 @@ const char *dsa_last_error(void);
  *   idx   [B, Lq, k] int32 (written)
  * Supported: H_I in {4, 8, 16, 32, 64}; d_I in {32, 64, 128}; 1 <= k <= 2048;
  * B >= 1; Lq >= 1; start_pos >= 0; start_pos + Lq - 1 <= Lk.
+ * When every row sees at most k positions (start_pos + Lq - 1 <= k), TopK
+ * keeps all of them: the rows are written directly and q_idx, k_idx and w
+ * are not read (the short-prefill case, where the selection equals the
+ * causal mask of dense attention).
  * Workspace: dsa_indexer_topk_workspace() bytes, contents undefined on entry. */
 size_t dsa_indexer_topk_workspace(int B, int Lq, int Lk, int start_pos, int H_I,
                                   int d_I, int k);

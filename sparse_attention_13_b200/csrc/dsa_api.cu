@@ -156,6 +156,20 @@ __global__ void check_indices_kernel(const int32_t* __restrict__ idx, int Lq, in
   if (__any_sync(0xffffffffu, bad) && threadIdx.x == 0) atomicAdd(bad_rows, 1);
 }
 
+// Index rows when every row sees at most k positions (t <= k): TopK keeps
+// all of P_t = {s : 0 <= s < t} ([IDX] §1, §4), so row t is 0, 1, ..., t-1
+// and then -1, and no score needs computing.  This is the short-prefill case
+// in which a sparse layer reads exactly what masked dense attention reads.
+__global__ void full_visible_rows_kernel(int32_t* __restrict__ idx, int64_t n, int Lq, int start_pos, int k) {
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = e / k;
+    const int r = static_cast<int>(e % k);
+    const int t = start_pos + static_cast<int>(row % Lq);
+    idx[e] = r < t ? r : -1;
+  }
+}
+
 }  // namespace dsa
 
 using namespace dsa;
@@ -202,6 +216,17 @@ dsa_status dsa_indexer_topk(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const 
   dsa_status st = check_indexer_args(q_idx, k_idx, w, B, Lq, Lk, start_pos, H_I, d_I, k, idx);
   if (st != DSA_OK) return st;
   if (!ws || !aligned16(ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_indexer_topk: null or misaligned workspace");
+  if (static_cast<long long>(start_pos) + Lq - 1 <= k) {
+    const int64_t n = static_cast<int64_t>(B) * Lq * k;
+    const int sms = device_sm_count();
+    if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
+    const unsigned blocks = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 8ll * sms)));
+    full_visible_rows_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(idx, n, Lq, start_pos, k);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("index rows launch: ") + cudaGetErrorString(e));
+    g_indexer_launches.fetch_add(1);
+    return DSA_OK;
+  }
   st = indexer_topk_launch(q_idx, k_idx, w, B, Lq, Lk, start_pos, H_I, d_I, k, idx, ws, ws_bytes,
                            static_cast<cudaStream_t>(stream));
   if (st == DSA_OK) g_indexer_launches.fetch_add(1);

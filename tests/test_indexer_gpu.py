@@ -75,7 +75,7 @@ def test_tiny_config_float_near_ties(dsa, oracle_mod):
 @pytest.mark.parametrize("B,L,H,d,kk", [
     (2, 1000, 64, 128, 256),    # ragged length, several 128-key tiles, compactions
     (1, 777, 16, 64, 100),      # odd k
-    (1, 300, 64, 128, 2048),    # t < k everywhere: every visible position, -1 padding
+    (1, 300, 64, 128, 2048),    # t <= k everywhere: rows written without scoring
     (3, 130, 32, 32, 7),        # tiny k, batch > 1, 64B swizzle
     (1, 2100, 8, 128, 64),      # many compactions per row (cap = 2k + 128)
 ])
@@ -134,13 +134,13 @@ def test_deterministic_reruns(dsa):
     (5, 20000, 20000, 64, 128, 2048),   # one query row per sequence at t = Lk
     (3, 9001, 7777, 32, 64, 300),       # t < Lk: the tail of the cache is not visible
     (2, 2100, 2100, 16, 128, 2048),     # T barely above k
-    (2, 1500, 1500, 64, 64, 2048),      # T < k: every visible position, -1 padding
-    (4, 130, 1, 16, 64, 5),             # T = 1: only position 0
+    (2, 1500, 1500, 64, 64, 2048),      # T <= k: every visible position, no scoring
+    (4, 130, 1, 16, 64, 5),             # T = 1: only position 0 (no scoring)
     (1, 50000, 49999, 64, 128, 1),      # k = 1
 ])
 def test_decode_rows_integer_exact(dsa, oracle_mod, B, Lk, start_pos, H, d, kk):
-    # Lq = 1 rows take the decode path (streamed score keys + cluster radix
-    # select); integer inputs make every score exact.
+    # Lq = 1 rows with T > k take the decode path (streamed score keys +
+    # cluster radix select); integer inputs make every score exact.
     q, k, w = indexer_inputs_host(Lk + H + kk, B, 1, Lk, H, d)
     got = _run(dsa, q, k, w, kk, start_pos=start_pos)
     for b in range(B):

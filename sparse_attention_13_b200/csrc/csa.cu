@@ -135,6 +135,7 @@ extern "C" {
 
 size_t dsa_csa_indexer_topk_workspace(int B, int Lq, int N_cmp, int start_pos, int m, int H_I, int d_I, int k) {
   if (B < 1 || Lq < 1 || N_cmp < 1 || start_pos < 0 || m < 1 || k < 1) return 0;
+  if (static_cast<long long>(B) * m > 2147483647ll) return 0;
   return csa_plan(B, Lq, N_cmp, start_pos, m, H_I, d_I, k).total;
 }
 

@@ -217,6 +217,72 @@ def csa_attn_row(q_row, c_cmp, idx, scale: float, Dv: int | None = None):
     return sparse_attn_row(q_row, c_cmp, c_cmp, idx, scale, Dv)
 
 
+# Low-precision selector ([IDX] §5.4).  Element formats from the OCP 8-bit
+# Floating Point (OFP8) and Microscaling (MX) v1.0 specifications:
+# (mantissa bits, exponent of the smallest normal, largest exponent, largest
+# finite value).
+_LP_FORMATS = {"e4m3": (3, -6, 8, 448.0), "e2m1": (1, 0, 2, 6.0)}
+
+
+def round_to_format(v, fmt: str) -> np.ndarray:
+    """Rounds float64 values to the E4M3 or E2M1 element grid: nearest, ties to
+    even, with subnormals below the smallest normal, saturating at the largest
+    finite value (E4M3 keeps its top code for NaN, so 448 is the largest).
+    Signs, including -0, are kept."""
+    m, emin, _, vmax = _LP_FORMATS[fmt]
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), emin)
+    ulp = np.exp2(e - m)
+    q = np.minimum(np.round(a / ulp) * ulp, vmax)     # np.round: half to even
+    return np.copysign(q, v)
+
+
+def mx_quantize(x, fmt: str, block: int = 32) -> np.ndarray:
+    """MX block quantization along the last axis: every run of `block`
+    consecutive elements shares the power-of-two scale
+    X = 2^(floor(log2 amax) - emax_elem) (emax_elem = 8 for E4M3, 2 for E2M1)
+    and each element becomes round_to_format(x / X).  Returns the values the
+    format represents, X * element, in float64.  (The 8-bit scale's range
+    limits of +-127 are not reached by these inputs and are not modelled.)"""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    assert d % block == 0
+    xb = x.reshape(x.shape[:-1] + (d // block, block))
+    amax = np.abs(xb).max(axis=-1, keepdims=True)
+    X = np.exp2(np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - _LP_FORMATS[fmt][2])
+    return (round_to_format(xb / X, fmt) * X).reshape(x.shape)
+
+
+def bf16_round(x) -> np.ndarray:
+    """Rounds float64 values first to float32 and then to bfloat16 (each to
+    nearest, ties to even): a score "quantised from FP32 to BF16".  Finite
+    inputs; returns float64."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _bf16_values(a) -> np.ndarray:
+    u = _bits(a).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def lowprec_indexer_row(q_row, k, w_row, T: int, fmt: str) -> np.ndarray:
+    """[IDX] §5.4: the §4 index score with the QK path in a low-precision
+    format and the score quantised from FP32 to BF16.  q_row [H, d] and the
+    keys are MX-quantised to `fmt` along d (blocks of 32), the head dots are
+    formed exactly from the quantised values (a tensor-core product
+    accumulates them in fp32), I = sum_j w_j ReLU(dot_j), and I is rounded to
+    bf16.  q_row, k as bf16 bits; w_row float32.  Returns [T] float64."""
+    qh = mx_quantize(_bf16_values(q_row), fmt)
+    kh = mx_quantize(_bf16_values(k)[:T], fmt) if T > 0 else np.zeros((0, qh.shape[1]))
+    w = np.asarray(w_row, dtype=np.float32).astype(np.float64)
+    I = np.maximum(kh @ qh.T, 0.0) @ w
+    return bf16_round(I)
+
+
 def _ptr_array(arrs):
     arr = (ctypes.c_void_p * len(arrs))()
     for i, a in enumerate(arrs):

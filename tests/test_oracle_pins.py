@@ -495,3 +495,94 @@ def test_csa_attention_reads_selected_compressed_entries(oracle_mod):
     out, lse = oracle_mod.csa_attn_row(q, C, np.array([3, -1, -1], np.int32), 0.5, Dv=8)
     np.testing.assert_allclose(out, np.broadcast_to(f32(C)[3, :8], out.shape), rtol=1e-15)
     np.testing.assert_allclose(lse, 0.5 * f32(q) @ f32(C)[3], rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# low-precision selector: MX-quantised QK path, scores rounded to bf16
+
+
+def test_e2m1_rounding_table(oracle_mod):
+    # the E2M1 grid is {0, 0.5, 1, 1.5, 2, 3, 4, 6}; midpoints go to the even
+    # code, anything beyond 6 saturates
+    x = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, 0.5, 3.0, -1.75, -0.0]
+    want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, 0.5, 3.0, -2.0, -0.0]
+    got = oracle_mod.round_to_format(x, "e2m1")
+    np.testing.assert_array_equal(got, want)
+    assert math.copysign(1.0, got[-1]) == -1.0
+
+
+def test_e4m3_rounding_table(oracle_mod):
+    x = [448.0, 460.0, 1e6, 2.0 ** -9, 2.0 ** -10, 1.5 * 2.0 ** -10, 0.3, 17.0, 19.0, 2.0 ** -6, 240.0, 232.0]
+    want = [448.0, 448.0, 448.0, 2.0 ** -9, 0.0, 2.0 ** -9, 0.3125, 16.0, 20.0, 2.0 ** -6, 240.0, 224.0]
+    np.testing.assert_array_equal(oracle_mod.round_to_format(x, "e4m3"), want)
+    # the positive finite E4M3 codes: 7 subnormals m 2^-9 and (1 + m/8) 2^(e-7)
+    # for e = 1..15, without the top code of e = 15 (NaN): 126 values
+    codes = sorted({m * 2.0 ** -9 for m in range(1, 8)} |
+                   {(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)} - {480.0})
+    assert len(codes) == 126 and codes[-1] == 448.0
+    np.testing.assert_array_equal(oracle_mod.round_to_format(codes, "e4m3"), codes)
+    image = np.unique(oracle_mod.round_to_format(np.geomspace(2.0 ** -12, 470.0, 200001), "e4m3"))
+    np.testing.assert_array_equal(image, [0.0] + codes)
+    # midpoints between neighbouring codes go to the one with the even mantissa
+    mids = (np.array(codes[:-1]) + np.array(codes[1:])) / 2
+    got = oracle_mod.round_to_format(mids, "e4m3")
+    lo, hi = np.array(codes[:-1]), np.array(codes[1:])
+    even_lo = np.array([round(c / 2.0 ** (max(math.floor(math.log2(c)), -6) - 3)) % 2 == 0 for c in lo])
+    np.testing.assert_array_equal(got, np.where(even_lo, lo, hi))
+    v = np.sort(np.random.default_rng(0).normal(scale=50, size=5000))
+    assert np.all(np.diff(oracle_mod.round_to_format(v, "e4m3")) >= 0)
+
+
+def test_mx_block_scale_rule(oracle_mod):
+    # amax = 1 gives X = 2^-8 for E4M3 (1.0 is element 256) and 2^-2 for E2M1
+    x = np.zeros(32)
+    x[0], x[1], x[2] = 1.0, 1e-6, -0.7
+    e4 = oracle_mod.mx_quantize(x, "e4m3")
+    assert e4[0] == 1.0 and e4[1] == 0.0           # 1e-6 * 256 lies below 2^-10
+    assert e4[2] == oracle_mod.round_to_format(-0.7 * 256, "e4m3") / 256
+    e2 = oracle_mod.mx_quantize(x, "e2m1")
+    assert e2[0] == 1.0 and e2[2] == -0.75          # -2.8 -> -3 on the E2M1 grid, times 2^-2
+    # blocks are independent: a large value in block 1 leaves block 0 alone
+    y = np.concatenate([x, 1000.0 * np.ones(32)])
+    np.testing.assert_array_equal(oracle_mod.mx_quantize(y, "e4m3")[:32], e4)
+    # integers in [-4, 4] are represented exactly in both formats
+    ints = np.random.default_rng(1).integers(-4, 5, size=(3, 128)).astype(float)
+    for fmt in ("e4m3", "e2m1"):
+        np.testing.assert_array_equal(oracle_mod.mx_quantize(ints, fmt), ints)
+
+
+def test_bf16_round(oracle_mod):
+    got = oracle_mod.bf16_round([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -3.0, 257.0, 259.0, 2.0 ** 17 + 512])
+    np.testing.assert_array_equal(got, [1.0, 1 + 2.0 ** -6, -3.0, 256.0, 260.0, 2.0 ** 17])
+
+
+def test_lowprec_selector_on_integer_inputs(oracle_mod):
+    # integer q, k lose nothing in either format, so the low-precision score is
+    # the exact score rounded to bf16; many scores then tie and the lower
+    # position wins
+    rng = np.random.default_rng(2)
+    H, d, T, k = 4, 64, 300, 40
+    q = bf16(rng.integers(-4, 5, size=(H, d)))
+    kk = bf16(rng.integers(-4, 5, size=(T, d)))
+    w = (2.0 ** -rng.integers(0, 3, size=H) * rng.choice([-1, 1], size=H)).astype(np.float32)
+    I = oracle_mod.indexer_row(q, kk, w, T)
+    for fmt in ("e4m3", "e2m1"):
+        Ilp = oracle_mod.lowprec_indexer_row(q, kk, w, T, fmt)
+        np.testing.assert_array_equal(Ilp, oracle_mod.bf16_round(I))
+    sel = oracle_mod.topk_row(Ilp, T, k)
+    want = sorted(sorted(range(T), key=lambda s: (-Ilp[s], s))[:k])
+    assert sel.tolist() == want
+    assert 0.0 <= oracle_mod.recall_row(oracle_mod.topk_row(I, T, k), sel) <= 1.0
+
+
+def test_lowprec_selector_recall_falls_with_precision(oracle_mod):
+    # normal inputs: E4M3 keeps more of the exact selection than E2M1
+    rng = np.random.default_rng(3)
+    H, d, T, k = 8, 128, 2000, 128
+    q = bf16(rng.normal(size=(H, d)))
+    kk = bf16(rng.normal(size=(T, d)))
+    w = rng.uniform(0.5, 1.5, size=H).astype(np.float32)
+    exact = oracle_mod.topk_row(oracle_mod.indexer_row(q, kk, w, T), T, k)
+    r = {fmt: oracle_mod.recall_row(exact, oracle_mod.topk_row(
+        oracle_mod.lowprec_indexer_row(q, kk, w, T, fmt), T, k)) for fmt in ("e4m3", "e2m1")}
+    assert 0.5 < r["e2m1"] < r["e4m3"] <= 1.0

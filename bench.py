@@ -227,6 +227,46 @@ def indexer_pairs(Lq, start_pos, B=1):
 
 
 # ----------------------------------------------------------------- GPU arm
+def time_stack(torch, dsa, stream, pat, layer_in, idx, ws, k, scale, D_v, steps, warmup, start_pos=0):
+    """Runs the layer loop `pat` eagerly through the C ABI (indexer on F
+    layers, attention on every layer) with CUDA events around each launch.
+    layer_in[l] holds q, kv, out and, on F layers, q_idx, k_idx, w.  Returns
+    (ms per step over `steps` timed steps, mean indexer ms per launch, mean
+    attention ms per launch, indexer ms per step)."""
+    def step(ev=None):
+        for l, role in enumerate(pat):
+            t = layer_in[l]
+            if role == "F":
+                if ev is not None:
+                    ev["idx"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                    ev["idx"][-1][0].record(stream)
+                dsa.indexer_topk(t["q_idx"], t["k_idx"], t["w"], k, start_pos=start_pos, out=idx, ws=ws)
+                if ev is not None:
+                    ev["idx"][-1][1].record(stream)
+            if ev is not None:
+                ev["attn"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
+                ev["attn"][-1][0].record(stream)
+            dsa.sparse_attn(t["q"], t["kv"], t["kv"], idx, scale, D_v=D_v, start_pos=start_pos, out=t["out"], ws=ws)
+            if ev is not None:
+                ev["attn"][-1][1].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = {"idx": [], "attn": []}
+    t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    t0.record(stream)
+    for _ in range(steps):
+        step(ev)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dsa.check_device_errors()
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["idx"]) if ev["idx"] else 0.0
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["attn"])
+    idx_per_step = sum(a.elapsed_time(b) for a, b in ev["idx"]) / steps
+    return t0.elapsed_time(t1) / steps, idx_ms, attn_ms, idx_per_step
+
+
 def run_dsa(args):
     import torch
     import torch.distributed as dist
@@ -332,6 +372,50 @@ def run_dsa(args):
         attn_flops=attn_flops, idx_flops=idx_flops, clocks=clk,
         launches=args.steps * (nF + len(pat)))
 
+    # The ratio sweep of the long prefill (1/1 and 1/2 beside the 1/4 stack
+    # timed above): the same 16 layers and shapes, with an indexer on every
+    # layer, or on every other layer.  Extra F layers get their own indexer
+    # inputs.  Kernels are warm; one warm-up step and a short timed region.
+    sweep = {}
+    if not args.no_sweep:
+        extra = []
+        for l in range(len(pat)):
+            if l not in q_idx:
+                q_idx[l] = torch.empty((1, L, P["H_I"], P["d_I"]), dtype=bf, device=dev)
+                k_idx[l] = torch.empty((1, L, P["d_I"]), dtype=bf, device=dev)
+                w[l] = torch.empty((1, L, P["H_I"]), dtype=f32, device=dev)
+                synth.fill_cuda(q_idx[l], seed, synth.Q_IDX, synth.INT9, l)
+                synth.fill_cuda(k_idx[l], seed, synth.K_IDX, synth.INT9, l)
+                synth.fill_cuda(w[l], seed, synth.W, synth.POW2W, l)
+                extra.append(l)
+        sw_steps = max(1, min(args.steps, 2))
+        runs = {}
+        for ratio in (1, 2):
+            spat = pattern_of(P["layers"], ratio)
+            lin = [dict(q=q, kv=kv[l], out=out, q_idx=q_idx.get(l), k_idx=k_idx.get(l), w=w.get(l))
+                   for l in range(len(spat))]
+            barrier()
+            runs[ratio] = (spat,) + time_stack(torch, dsa, stream, spat, lin, idx, ws, k, scale, P["D_v"],
+                                               sw_steps, 1)
+        runs[P["ratio"]] = (pat, ms, idx_ms, attn_ms, idx_ms * nF)
+        all_f_idx = runs[1][4]
+        for ratio in sorted(runs):
+            spat, sms, sidx, sattn, sidx_step = runs[ratio]
+            sms = max_over_ranks(sms)
+            m = spat.count("F")
+            sweep[f"1/{ratio}"] = dict(
+                pattern=spat, ms_per_step=sms, tokens_per_s=job_rate(L, world, sms),
+                indexer_ms_per_step=sidx_step, attn_ms_per_step=sattn * len(spat),
+                indexer_share=sidx_step / (sidx_step + sattn * len(spat)),
+                indexer_ms_expected=m / len(spat) * all_f_idx,
+                indexer_launches_per_step=m,
+                steps=sw_steps if ratio != P["ratio"] else args.steps,
+                warmup=1 if ratio != P["ratio"] else args.warmup)
+        for l in extra:
+            del q_idx[l], k_idx[l], w[l]
+        torch.cuda.empty_cache()
+    result["prefill"]["sweep"] = sweep
+
     # e2e through the public API with host buffers
     host_in = []
     for l in sorted(q_idx):
@@ -429,7 +513,8 @@ def run_dsa(args):
     d_idx_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["idx"])
     d_attn_ms = statistics.mean(a.elapsed_time(b) for a, b in dev_ev["attn"])
     # the timed decode step is one CUDA graph of the whole 48-layer step (the
-    # way a decode loop replays it); ~0.5 s of replays so the clocks are sampled
+    # way a decode loop replays it); several seconds of replays, so that the
+    # clock record holds many samples
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
@@ -443,7 +528,7 @@ def run_dsa(args):
         graph.replay()
     torch.cuda.synchronize(dev)
     dsa.check_device_errors()
-    dsteps = 200
+    dsteps = args.decode_steps
     barrier()
     torch.cuda.synchronize(dev)
     dclocks = ClockSampler(uuid)
@@ -502,11 +587,106 @@ def run_dsa(args):
                                  "d2h_bytes_per_step": hout.numel() * 2})
     # per step: score + top-k kernels per F layer, attention + split merge per layer
     result["decode"]["launches"] = dsteps * (2 * nFd + 2 * len(dpat))
+    del dq_idx, dk_idx, dw, dq, dkv, dset, dset_out, dset_layers, dh2d_pairs, dd2h_pairs, hq, hqi, hw, hout
+    torch.cuda.empty_cache()
+    if not args.no_sweep:
+        result["config2"] = run_config2(torch, dsa, synth, dev, stream, seed, max_over_ranks)
+        result["config3"] = run_config3(torch, dsa, synth, dev, stream, seed, max_over_ranks, world, barrier)
     result["peaks"] = (hbm_peak, tc_peak, peak_kind)
     result["world"] = world
     if world > 1:
         dist.destroy_process_group()
     return result
+
+
+CONFIG2 = dict(B=1, L=16384, H_I=64, d_I=128, k=2048)
+CONFIG3 = dict(B=1, L=32768, pattern="FSSSFSSS", H_I=64, d_I=128, k=2048, n_h=128, D_qk=576, D_v=512)
+
+
+def run_config2(torch, dsa, synth, dev, stream, seed, max_over_ranks, reps=20):
+    """One F layer's indexer + top-k alone (B = 1, L = 16,384, 64 heads x 128,
+    k = 2048, integer inputs), `reps` launches after 3 warm-up launches.  The
+    kernel is timed on its own, so its roofline uses the burst bf16 peak."""
+    C = CONFIG2
+    L = C["L"]
+    qi = torch.empty((1, L, C["H_I"], C["d_I"]), dtype=torch.bfloat16, device=dev)
+    ki = torch.empty((1, L, C["d_I"]), dtype=torch.bfloat16, device=dev)
+    wi = torch.empty((1, L, C["H_I"]), dtype=torch.float32, device=dev)
+    synth.fill_cuda(qi, seed + 2, synth.Q_IDX, synth.INT9, 0)
+    synth.fill_cuda(ki, seed + 2, synth.K_IDX, synth.INT9, 0)
+    synth.fill_cuda(wi, seed + 2, synth.W, synth.POW2W, 0)
+    out = torch.empty((1, L, C["k"]), dtype=torch.int32, device=dev)
+    ws = torch.empty(dsa.indexer_topk_workspace(1, L, L, 0, C["H_I"], C["d_I"], C["k"]), dtype=torch.uint8,
+                     device=dev)
+    for _ in range(3):
+        dsa.indexer_topk(qi, ki, wi, C["k"], out=out, ws=ws)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    t0.record(stream)
+    for _ in range(reps):
+        dsa.indexer_topk(qi, ki, wi, C["k"], out=out, ws=ws)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dsa.check_device_errors()
+    ms = max_over_ranks(t0.elapsed_time(t1) / reps)
+    flops = indexer_pairs(L, 0) * 2 * C["H_I"] * C["d_I"]
+    burst = measured_burst_tflops()
+    return {"workload": f"B=1, L={L}, one F layer (indexer + top-k), H_I=64 d_I=128 k=2048, integer "
+                        "q/k in [-4,4], w = +-2^-m", "ms_per_launch": ms, "launches": reps,
+            "roofline": {"bound": "tensor", "kernel": "indexer_topk", "achieved": flops / ms / 1e9,
+                         "peak": burst[0], "unit": "TFLOP/s", "frac": flops / ms / 1e9 / burst[0],
+                         "peak_kind": f"{burst[1]} bf16 burst (kernel timed alone)",
+                         "per_launch_flops": flops}}
+
+
+def run_config3(torch, dsa, synth, dev, stream, seed, max_over_ranks, world, barrier, steps=5):
+    """The eight-layer FSSSFSSS stack (B = 1, L = 32,768, k = 2048, MLA 128
+    heads 576/512, correlated layers), `steps` timed steps after 3 warm-up
+    steps.  Each layer has its own query and latent cache; the layers share
+    one output buffer."""
+    C = CONFIG3
+    L, pat = C["L"], C["pattern"]
+    bf = torch.bfloat16
+    lin = []
+    out = torch.empty((1, L, C["n_h"], C["D_v"]), dtype=bf, device=dev)
+    for l, role in enumerate(pat):
+        t = dict(q=torch.empty((1, L, C["n_h"], C["D_qk"]), dtype=bf, device=dev),
+                 kv=torch.empty((1, L, C["D_qk"]), dtype=bf, device=dev), out=out)
+        synth.fill_cuda(t["q"], seed + 3, synth.Q, synth.NORMAL, l, sigma=0.5, corr=True)
+        synth.fill_cuda(t["kv"], seed + 3, synth.KV, synth.NORMAL, l, sigma=0.5, corr=True)
+        if role == "F":
+            t["q_idx"] = torch.empty((1, L, C["H_I"], C["d_I"]), dtype=bf, device=dev)
+            t["k_idx"] = torch.empty((1, L, C["d_I"]), dtype=bf, device=dev)
+            t["w"] = torch.empty((1, L, C["H_I"]), dtype=torch.float32, device=dev)
+            synth.fill_cuda(t["q_idx"], seed + 3, synth.Q_IDX, synth.INT9, l, corr=True)
+            synth.fill_cuda(t["k_idx"], seed + 3, synth.K_IDX, synth.INT9, l, corr=True)
+            synth.fill_cuda(t["w"], seed + 3, synth.W, synth.POW2W, l)
+        lin.append(t)
+    idx = torch.empty((1, L, C["k"]), dtype=torch.int32, device=dev)
+    dims = dsa.make_dims(B=1, Lq=L, Lk=L, start_pos=0, H_I=C["H_I"], d_I=C["d_I"], k=C["k"], n_h=C["n_h"],
+                         D_qk=C["D_qk"], D_v=C["D_v"], scale=1 / math.sqrt(C["D_qk"]), k_row_stride=C["D_qk"],
+                         v_row_stride=C["D_qk"])
+    ws = torch.empty(dsa.indexcache_forward_workspace(dims), dtype=torch.uint8, device=dev)
+    barrier()
+    ms, idx_ms, attn_ms, idx_step = time_stack(torch, dsa, stream, pat, lin, idx, ws, C["k"],
+                                               1 / math.sqrt(C["D_qk"]), C["D_v"], steps, 3)
+    ms = max_over_ranks(ms)
+    a_flops = attn_units(L, 0, C["k"]) * 2 * C["n_h"] * (C["D_qk"] + C["D_v"])
+    i_flops = indexer_pairs(L, 0) * 2 * C["H_I"] * C["d_I"]
+    return {"workload": f"B=1, L={L}, 8 layers {pat}, H_I=64 d_I=128 k=2048, MLA 128 heads 576/512, "
+                        "correlated layers", "ms_per_step": ms, "tokens_per_s": job_rate(L, world, ms),
+            "steps": steps, "warmup": 3, "indexer_ms": idx_ms, "attn_ms": attn_ms,
+            "indexer_share": idx_step / ms,
+            "attn_tflops": a_flops / attn_ms / 1e9, "indexer_tflops": i_flops / idx_ms / 1e9,
+            "step_flops": 2 * i_flops + 8 * a_flops}
+
+
+def measured_burst_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f).get("bf16_tflops", 1590.0), "measured"
+    return 1590.0, "fallback"
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -522,6 +702,70 @@ def _oracle_keys(seed, B, L, d):
     if key not in _ORACLE_KEYS:
         _ORACLE_KEYS[key] = synth.rows(seed, synth.K_IDX, synth.INT9, 0, (B, L, d), np.arange(L))
     return _ORACLE_KEYS[key]
+
+
+def _par_init():
+    import oracle
+    oracle.build()
+    _oracle_keys(SEED, 1, PREFILL["L"], PREFILL["d_I"])
+
+
+def _par_indexer_row(t):
+    """One oracle indexer + top-k row of the prefill stack (worker process)."""
+    import numpy as np
+
+    import oracle
+    from sparse_attention_13_b200 import synth
+    P = PREFILL
+    k_h = _oracle_keys(SEED, 1, P["L"], P["d_I"])
+    qr = synth.rows(SEED, synth.Q_IDX, synth.INT9, 0, (1, P["L"], P["H_I"], P["d_I"]),
+                    np.arange(P["H_I"]) + t * P["H_I"])
+    wr = synth.rows(SEED, synth.W, synth.POW2W, 0, (1, P["L"], P["H_I"]), [t], bf16=False)[0]
+    return oracle.topk_row(oracle.indexer_row(qr, k_h, wr, t), t, P["k"])
+
+
+def _par_attn_row(args):
+    """One oracle attention row of the prefill stack (worker process)."""
+    import numpy as np
+
+    import oracle
+    from sparse_attention_13_b200 import synth
+    t, sel = args
+    P = PREFILL
+    valid = sel[sel >= 0]
+    rows_kv = synth.rows(SEED, synth.KV, synth.NORMAL, 0, (1, P["L"], P["D_qk"]), valid, sigma=0.5)
+    q_r = synth.rows(SEED, synth.Q, synth.NORMAL, 0, (1, P["L"], P["n_h"], P["D_qk"]),
+                     np.arange(P["n_h"]) + t * P["n_h"], sigma=0.5)
+    a = time.perf_counter()
+    oracle.sparse_attn_row(q_r, rows_kv, rows_kv, np.arange(len(valid), dtype=np.int32),
+                           1 / math.sqrt(P["D_qk"]), Dv=P["D_v"])
+    return time.perf_counter() - a
+
+
+def oracle_parallel_sample(procs):
+    """The same oracle routines run row-parallel: `procs` spawned processes
+    (one single-threaded oracle each), one stratified indexer row and one
+    attention row per process; wall time of each batch, extrapolated to the
+    stack like the single-threaded sample."""
+    import multiprocessing as mp
+    P = PREFILL
+    L = P["L"]
+    nF = pattern_of(P["layers"], P["ratio"]).count("F")
+    ts = [int(L * (2 * j + 1) / (2 * procs)) for j in range(procs)]
+    with mp.get_context("spawn").Pool(procs, initializer=_par_init) as pool:
+        pool.map(_par_indexer_row, [1] * procs, chunksize=1)   # workers up, keys built
+        a = time.perf_counter()
+        sels = pool.map(_par_indexer_row, ts, chunksize=1)
+        w_idx = time.perf_counter() - a
+        a = time.perf_counter()
+        pool.map(_par_attn_row, list(zip(ts, sels)), chunksize=1)
+        w_attn = time.perf_counter() - a
+    per_tok = nF * w_idx / procs + P["layers"] * w_attn / procs
+    return {"value": 1.0 / per_tok, "unit": "tokens/s", "processes": procs,
+            "kind": "oracle, row-parallel",
+            "sample": f"{procs} spawned single-threaded oracle processes, one indexer row each at "
+                      f"stratified t, then one attention row each; wall time per batch, extrapolated "
+                      f"by rows x layers", "seconds": w_idx + w_attn}
 
 
 def oracle_sample(budget_rows=4, decode=True):
@@ -609,7 +853,8 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": config_of(args.gpus),
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count() or 1,
+                             "kind": "oracle",
                              "sample": f"per step: 1 indexer row at t = L/2 (the mean causal row) and "
                                        f"1 attention row of the L = {P['L']} prefill stack, single host "
                                        f"thread, extrapolated to the 16-layer stack (prefill metric only)"},
@@ -847,6 +1092,10 @@ def main():
                     help="profiling: indexer|attn|decode_idx|decode_attn|decode_step; "
                          "quality runs the selection-quality tools, csa one CSA-style layer")
     ap.add_argument("--reps", type=int, default=2)
+    ap.add_argument("--decode-steps", type=int, default=2000,
+                    help="CUDA-graph replays in the decode timed region")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the ratio sweep and the config-2/config-3 lines (short runs)")
     args = ap.parse_args()
     if args.kernel_case == "quality":
         selection_quality(args.seq or 8192)
@@ -885,8 +1134,11 @@ def main():
                              "traffic": idx_tr, "per_launch_flops": pf["idx_flops"],
                              "avg_launch_ms": pf["idx_ms"]},
         "indexer_share": pf["indexer_share"],
+        "sweep": {"workload": "prefill B=1, L=200000, 16 layers, F ratios 1/1 (F x16), 1/2 (FS x8), "
+                              "1/4 (FSSS x4); indexer_ms_expected = M/N x the all-F indexer time per step",
+                  "ratios": pf["sweep"]},
         "decode": {"ms_per_step": dc["ms_per_step"], "higher_is_better": False,
-                   "timing": "CUDA graph of the 48-layer step, 200 replays",
+                   "timing": f"CUDA graph of the 48-layer step, {args.decode_steps} replays",
                    "gpu_launches": dc["launches"],
                    "idx_launch_ms": dc["idx_ms"], "attn_launch_ms": dc["attn_ms"],
                    "roofline": {"bound": "hbm", "achieved": dc["step_bytes"] / dc["ms_per_step"] / 1e6,
@@ -898,12 +1150,19 @@ def main():
         "gpu_launches": pf["launches"],
         "clocks": pf["clocks"],
     }
+    if "config2" in res:
+        line["config2"] = res["config2"]
+        line["config3"] = res["config3"]
     if world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample()
+        host_cores = os.cpu_count() or 1
         line["cpu_baseline"] = {"value": cb["prefill_tokens_per_s"], "unit": "tokens/s", "cores": 1,
+                                "host_cores": host_cores,
                                 "kind": "oracle", "sample": cb["sample"],
                                 "decode_ms_per_step": cb["decode_ms_per_step"],
                                 "decode_sample": cb["decode_sample"]}
+        if host_cores > 1:
+            line["cpu_baseline"]["row_parallel"] = oracle_parallel_sample(min(host_cores, 64))
     print(json.dumps(line), flush=True)
 
 

@@ -88,8 +88,14 @@ dsa_status dsa_indexer_topk(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
  * An empty set gives out = 0.  MLA ([IDX] §4): pass k = v = the latent cache
  * with row stride 576, D_qk = 576, D_v = 512 (V is the first 512 columns);
  * every query head reads the same latent row.  Index rows come from
- * dsa_indexer_topk (any order is accepted; -1 entries are skipped; valid
- * entries must satisfy 0 <= S_t[r] < t).
+ * dsa_indexer_topk (any order is accepted; -1 entries are skipped, and so
+ * are entries outside [0, Lk), which would name rows of another sequence or
+ * none; causal use needs 0 <= S_t[r] < t).
+ * Numerics: each score is an fp32 sum of exact bf16 products (the MLA kernel
+ * splits the 576 columns over two CTAs and adds their fp32 partial sums, so
+ * no intermediate is narrowed and no input range is imposed beyond finite
+ * fp32 scores); the softmax runs in fp32, the weights are rounded to bf16 for
+ * the P.V product (fp32 accumulation), the output to bf16.
  *   q   [B, Lq, n_h, D_qk] bf16
  *   kbuf rows: kbuf + (b*Lk + s)*k_row_stride, D_qk bf16 each
  *   vbuf rows: vbuf + (b*Lk + s)*v_row_stride, D_v bf16 each

@@ -19,11 +19,12 @@
 //                    a double-buffered S tile, then, one chunk behind,
 //                    O_c += P V_c with P read from TMEM and V_c the gathered
 //                    slabs 0..3 read as an MN-major B operand;
-//     4 sender warps (thread = head) read S_c as soon as QK completes, pack it
-//                    as fp16 and ship it to the peer with one bulk copy into
-//                    the peer's shared memory (tx-counted on its mbarrier);
-//                    they also load the next row's query into TMEM as soon as
-//                    the last QK of the current row has completed;
+//     4 sender warps (thread = head) read S_c as soon as QK completes and
+//                    store it, fp32, straight into the peer's shared memory
+//                    with asynchronous remote stores that count their bytes
+//                    on the peer's mbarrier; they also load the next row's
+//                    query into TMEM as soon as the last QK of the current row
+//                    has completed;
 //     8 softmax warps (thread = head = TMEM lane x half of the chunk) add the
 //                    peer's partial (S = S_0 + S_1, identical in both CTAs as
 //                    fp32 addition commutes), mask padded rows (fully valid
@@ -41,7 +42,6 @@
 // simt_sparse_attn_kernel: plain CUDA-core kernel for small head dims
 // (D_qk, D_v <= 128, separate K and V tensors), one block per query row.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cmath>
@@ -83,7 +83,7 @@ simt_sparse_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < nv; ++r) {
       const int s = irow[r];
-      if (s < 0) continue;
+      if (s < 0 || s >= Lk) continue;  // padding, or a position outside the sequence: skipped
       const __nv_bfloat16* kr = kbase + static_cast<int64_t>(s) * ks;
       float dot = 0.f;
       for (int c = lane; c < Dqk; c += 32) dot += qs[h * Dqk + c] * __bfloat162float(kr[c]);
@@ -119,7 +119,7 @@ constexpr int kSlabBytes = kChunk * 128;       // one 64-column slab of a chunk,
 constexpr int kMaxSlabs = 5;                   // CTA0: columns 0..255, CTA1: 256..575
 constexpr int kStageBytes = kMaxSlabs * kSlabBytes;
 constexpr int kStages = 3;
-constexpr int kXBytes = kNH * kChunk * 2;      // partial score tile, fp16
+constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile, fp32
 constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, bf16
 // TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64; P(c) overwrites
 // the first 32 columns of S(c) as bf16 pairs) | Q (bf16 pairs, 128)
@@ -131,7 +131,7 @@ constexpr int kMmaWarpA = 19;
 constexpr int kMlaThreads = 20 * 32;           // 20 warps: 96 registers per thread
 constexpr float kRescaleThresh = 8.0f;          // log2 units
 constexpr int kPairBarBase = 2;                 // named barriers 2..5 and 6..9: the two softmax warps of a quadrant
-constexpr int kSendBar = 10;                    // named barriers 10, 11: the sender warps
+constexpr int kSendBar = 10;                    // named barrier 10: the sender warps
 
 struct MlaBars {
   uint64_t kv_full[kStages], kv_empty[kStages];
@@ -146,8 +146,8 @@ struct MlaBars {
   int abort_flag;
 };
 
-// shared memory: gather ring | peer partials X_in[2] | own partials X_out[2] | Q rope
-constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 4 * kXBytes + kQRopeBytes +
+// shared memory: gather ring | peer partials X_in[2] (fp32) | Q rope
+constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kQRopeBytes +
                          static_cast<int>(sizeof(MlaBars)) + 64;
 
 struct MlaParams {
@@ -188,8 +188,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* kv_smem = smem;
   uint8_t* xin_smem = kv_smem + kStages * kStageBytes;   // X_in[2]: the peer's partials
-  uint8_t* xout_smem = xin_smem + 2 * kXBytes;           // X_out[2]: this CTA's partials
-  uint8_t* qrope_smem = xout_smem + 2 * kXBytes;         // CTA1: Q[:, 512:576]
+  uint8_t* qrope_smem = xin_smem + 2 * kXBytes;          // CTA1: Q[:, 512:576]
   MlaBars* bb = reinterpret_cast<MlaBars*>(qrope_smem + kQRopeBytes);
   volatile int* abort_flag = &bb->abort_flag;
 
@@ -371,8 +370,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int stid = threadIdx.x - kSendWarp0 * 32;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const uint32_t xin_remote = mapa_shared(smem_u32(xin_smem), peer);
-    const uint32_t xfull_remote[2] = {mapa_shared(smem_u32(&bb->x_full[0]), peer),
-                                      mapa_shared(smem_u32(&bb->x_full[1]), peer)};
+    // x_full[0] and x_full[1] are adjacent: the peer's x_full[sb] is at + 8 sb
+    const uint32_t xfull_remote = mapa_shared(smem_u32(&bb->x_full[0]), peer);
     // A failed (timed-out) wait only clears `ok`; the sender warps leave their
     // loops together, at the next named barrier, so none is left waiting there.
     uint32_t g = 0, it_n = 0;
@@ -424,54 +423,38 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const int sb = g & 1;
         if (c == c_pf && nq != nullptr)
           for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
-        if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag));
+        // the peer's X_in[sb] is free once its softmax has consumed chunk g-2
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_free[sb], ((g >> 1) & 1) ^ 1, abort_flag));
         tc_fence_after();
-        uint32_t hv[32];
         if (ok) {
-          uint32_t v[32];
-          tmem_ld32<32>(t_lane + kSCol + sb * 64, v);
-          tmem_ld_wait();
+          // this CTA's X_in[sb] receives the peer's partial of chunk g: one
+          // arrival plus its bytes complete the phase
+          if (stid == 0) mbar_arrive_expect_tx(&bb->x_full[sb], kXBytes);
+          // row h of the peer's tile, 16-byte pieces XOR-swizzled by h & 7 so
+          // that the peer's per-head reads are free of bank conflicts: piece j
+          // of the row sits at byte offset off ^ (j << 4) of X_in (bits 4..7 of
+          // off are h & 7 and zero above, for j < 16)
+          const uint32_t off = sb * kXBytes + h * 256 + ((h & 7) << 4);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) hv[j] = pack_half2_sat(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-          tmem_ld32<32>(t_lane + kSCol + sb * 64 + 32, v);
-          tmem_ld_wait();
+          for (int hv = 0; hv < 4; ++hv) {
+            uint32_t v[16];
+            tmem_ld32<16>(t_lane + kSCol + sb * 64 + hv * 16, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) hv[16 + j] = pack_half2_sat(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+            for (int j = 0; j < 4; ++j)
+              st_async_v4(xin_remote + (off ^ ((4 * hv + j) << 4)), v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                          v[4 * j + 3], xfull_remote + 8 * sb);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(&bb->s_read[sb]);
-        // X_out[sb] was last read by the DMA of chunk g-2
-        if (stid == 0) bulk_wait_read_allbut1();
-        ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
-        if (!ok) break;
-        {
-          uint8_t* xo = xout_smem + sb * kXBytes + h * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(xo + ((j ^ (h & 7)) << 4)) =
-                make_uint4(hv[4 * j], hv[4 * j + 1], hv[4 * j + 2], hv[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(kSendBar + 1, kSendWarps * 32);
-        if (stid == 0) {
-          // the peer consumed its X_in[sb] from chunk g-2; this CTA expects
-          // the peer's partial of chunk g in its own X_in[sb]
-          if (mbar_wait_cluster(&bb->x_free[sb], ((g >> 1) & 1) ^ 1, abort_flag)) {
-            mbar_arrive_expect_tx(&bb->x_full[sb], kXBytes);
-            bulk_copy_to_peer(xin_remote + sb * kXBytes, smem_u32(xout_smem + sb * kXBytes), kXBytes,
-                              xfull_remote[sb]);
-            bulk_commit_group();
-          } else {
-            ok = false;  // the abort flag is raised; the next barrier ends the loop
-          }
-        }
       }
       ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
       if (!ok) break;
       ++it_n;
     }
-    if (stid == 0) bulk_wait_read_all();  // the last DMA has read X_out
   } else {
     // ------------------------------------------------------------ softmax
     // thread = (head h = TMEM lane, half hf of the chunk's 64 columns)
@@ -546,20 +529,17 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
 #pragma unroll
           for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
         }
-        // + the peer's partial scores of the same columns (fp16)
+        // + the peer's partial scores of the same columns (fp32)
         if (ok) ok = mbar_wait_cluster(&bb->x_full[sb], (g >> 1) & 1, abort_flag);
         if (ok) {
-          const uint8_t* xr = xin_smem + sb * kXBytes + h * 128;
+          const uint8_t* xr = xin_smem + sb * kXBytes + h * 256;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 o = *reinterpret_cast<const uint4*>(xr + (((hf * 4 + j) ^ (h & 7)) << 4));
-            const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
-              s[8 * j + 2 * e] += f.x;
-              s[8 * j + 2 * e + 1] += f.y;
-            }
+          for (int j = 0; j < 8; ++j) {
+            const float4 o = *reinterpret_cast<const float4*>(xr + (((hf * 8 + j) ^ (h & 7)) << 4));
+            s[4 * j] += o.x;
+            s[4 * j + 1] += o.y;
+            s[4 * j + 2] += o.z;
+            s[4 * j + 3] += o.w;
           }
         }
         // mask, scale, chunk max (combined with the other half of the head)

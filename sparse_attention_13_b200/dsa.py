@@ -158,8 +158,9 @@ NOALLOC_SCRATCH_BYTES = 72 * 1024 * 1024
 
 def indexer_topk_noalloc(q_idx, k_idx, w, k: int, *, start_pos: int = 0, out=None):
     """Same as indexer_topk, for callers that cannot hand the library a
-    workspace: the scratch comes from a fixed 48 MiB device array inside the
-    library (shared by every call; do not overlap calls on the GPU)."""
+    workspace: the scratch comes from a fixed device array of
+    NOALLOC_SCRATCH_BYTES inside the library (shared by every call; do not
+    overlap calls on the GPU)."""
     import torch
     B, Lq, H, d = q_idx.shape
     Lk = k_idx.shape[1]

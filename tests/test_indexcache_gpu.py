@@ -1,8 +1,10 @@
 """GPU parity of indexcache_forward (the F/S layer loop, through the C ABI)
-against the oracle's loop: the tiny FSFS stack in full, an FSSSFSSS MLA stack
-with correlated layers on sampled rows, the reuse identity of the IndexCache
-explainer (§1.1: S layers attend through the last F layer's indices with
-their own K/V) and the indexer launch count (two for FSSSFSSS)."""
+against the oracle's loop: the tiny FSFS stack in full, FSSSFSSS MLA stacks
+with correlated layers on sampled rows (L = 4,096, and the eight-layer stack
+at L = 32,768), four-layer FFFF and FSFS stacks at L = 200,000, the reuse
+identity of the IndexCache explainer (§1.1: S layers attend through the last
+F layer's indices with their own K/V) and the indexer launch count (two for
+FSSSFSSS)."""
 import math
 
 import numpy as np
@@ -152,3 +154,107 @@ def test_bounded_wait_expiry_reports_timeout_and_context_survives(dsa, oracle_mo
     for i in (0, 31, 32, 299):
         I = oracle_mod.indexer_row(q[0, i], k[0], w[0, i], i)
         check_topk_row(got[0, i], oracle_mod.topk_row(I, i, kk), I, kk)
+
+
+def _sampled_stack(dsa, oracle_mod, pattern, L, seed, rows, att_rows, corr, shared_q):
+    """Runs `pattern` through indexcache_forward at B = 1, length L, with the
+    MLA shape and k = 2048, and checks sampled rows against the oracle:
+      - the index cache after each F layer's segment, bit for bit (the segment
+        is run as a prefix of the pattern: the cache then holds that F layer's
+        selection);
+      - every layer's LSE, through the oracle's selection of the F layer that
+        governs it (the reuse rule of [IC] §1.1-§1.2);
+      - the last layer's output.
+    With shared_q every layer reads one query tensor and writes one output
+    buffer (the L = 200,000 stacks would not fit otherwise); the per-layer
+    LSE then checks each layer's attention."""
+    import torch
+    B, H, dI, k = 1, 64, 128, 2048
+    scale = 1 / math.sqrt(576)
+    kw = dict(sigma=0.5, corr=corr)
+    dl = []
+    q_shared = out_shared = None
+    if shared_q:
+        q_shared = torch.empty((B, L, 128, 576), dtype=torch.bfloat16, device="cuda")
+        synth.fill_cuda(q_shared, seed, synth.Q, synth.NORMAL, 0, sigma=0.5)
+        out_shared = torch.empty((B, L, 128, 512), dtype=torch.bfloat16, device="cuda")
+    for l, role in enumerate(pattern):
+        ent = dict(kbuf=torch.empty((B, L, 576), dtype=torch.bfloat16, device="cuda"),
+                   lse=torch.empty((B, L, 128), dtype=torch.float32, device="cuda"))
+        synth.fill_cuda(ent["kbuf"], seed, synth.KV, synth.NORMAL, l, **kw)
+        ent["vbuf"] = ent["kbuf"]
+        if shared_q:
+            ent["q"], ent["out"] = q_shared, out_shared
+        else:
+            ent["q"] = torch.empty((B, L, 128, 576), dtype=torch.bfloat16, device="cuda")
+            synth.fill_cuda(ent["q"], seed, synth.Q, synth.NORMAL, l, **kw)
+            ent["out"] = torch.empty((B, L, 128, 512), dtype=torch.bfloat16, device="cuda")
+        if role == "F":
+            ent["q_idx"] = torch.empty((B, L, H, dI), dtype=torch.bfloat16, device="cuda")
+            ent["k_idx"] = torch.empty((B, L, dI), dtype=torch.bfloat16, device="cuda")
+            ent["w"] = torch.empty((B, L, H), dtype=torch.float32, device="cuda")
+            synth.fill_cuda(ent["q_idx"], seed, synth.Q_IDX, synth.INT9, l, corr=corr)
+            synth.fill_cuda(ent["k_idx"], seed, synth.K_IDX, synth.INT9, l, corr=corr)
+            synth.fill_cuda(ent["w"], seed, synth.W, synth.POW2W, l)
+        dl.append(ent)
+    dims = dsa.make_dims(B=B, Lq=L, Lk=L, start_pos=0, H_I=H, d_I=dI, k=k, n_h=128, D_qk=576,
+                         D_v=512, scale=scale, k_row_stride=576, v_row_stride=576)
+    idx = torch.empty((B, L, k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(dsa.indexcache_forward_workspace(dims), dtype=torch.uint8, device="cuda")
+    f_layers = [l for l, r in enumerate(pattern) if r == "F"]
+    caches = {}
+    for F in f_layers:
+        # prefix up to F's segment end: the cache then holds F's selection
+        end = next((g for g in f_layers if g > F), len(pattern))
+        before = dsa.indexer_launch_count()
+        dsa.indexcache_forward(pattern[:end], dl[:end], dims, idx, ws=ws)
+        dsa.check_device_errors()
+        assert dsa.indexer_launch_count() - before == pattern[:end].count("F")
+        caches[F] = idx[0, rows].cpu().numpy()
+    lse_all = [dl[l]["lse"][0, att_rows].cpu().numpy() for l in range(len(pattern))]
+    out_last = dl[-1]["out"][0, att_rows].float().cpu().numpy()
+    sel = {}
+    for F in f_layers:
+        kh = synth.tensor(seed, synth.K_IDX, synth.INT9, F, (B, L, dI), corr=corr)
+        for n, i in enumerate(rows):
+            qr = synth.rows(seed, synth.Q_IDX, synth.INT9, F, (B, L, H, dI), np.arange(H) + H * i, corr=corr)
+            wr = synth.rows(seed, synth.W, synth.POW2W, F, (B, L, H), [i], bf16=False)[0]
+            I = oracle_mod.indexer_row(qr, kh[0], wr, i)
+            sel[F, i] = oracle_mod.topk_row(I, i, k)
+            np.testing.assert_array_equal(caches[F][n], sel[F, i])
+        del kh
+    gov = {}
+    for l, role in enumerate(pattern):
+        gov[l] = l if role == "F" else gov[l - 1]
+    for l in range(len(pattern)):
+        ql = 0 if shared_q else l
+        qkw = dict(sigma=0.5) if shared_q else kw
+        for n, i in enumerate(att_rows):
+            s_row = sel[gov[l], i]
+            valid = s_row[s_row >= 0]
+            qr = synth.rows(seed, synth.Q, synth.NORMAL, ql, (B, L, 128, 576), np.arange(128) + 128 * i, **qkw)
+            kr = synth.rows(seed, synth.KV, synth.NORMAL, l, (B, L, 576), valid.astype(np.uint64), **kw)
+            o, lse_o = oracle_mod.sparse_attn_row(qr, kr, kr, np.arange(len(valid), dtype=np.int32), scale, Dv=512)
+            fin = np.isfinite(lse_o)
+            assert np.array_equal(np.isfinite(lse_all[l][n]), fin)
+            np.testing.assert_allclose(lse_all[l][n][fin], lse_o[fin], rtol=0, atol=1e-5 + 2048 * 2.0 ** -24 + 3.6e-4)
+            if l == len(pattern) - 1:
+                _close(out_last[n], o)
+
+
+def test_config3_stack_fsssfsss_l32768(dsa, oracle_mod):
+    # The eight-layer FSSSFSSS stack at its stated size (B = 1, L = 32,768,
+    # k = 2048, correlated layers): the index cache after both F segments and
+    # every layer's attention on rows stratified over t.
+    _sampled_stack(dsa, oracle_mod, "FSSSFSSS", 32768, 61,
+                   rows=[1, 2047, 2048, 2049, 16384, 32767], att_rows=[1, 2048, 20001, 32767],
+                   corr=True, shared_q=False)
+
+
+@pytest.mark.parametrize("pattern", ["FFFF", "FSFS"])
+def test_long_stacks_l200k(dsa, oracle_mod, pattern):
+    # Four-layer stacks of the 1/1 and 1/2 patterns at L = 200,000 (the long
+    # prefill of the sweep), uncorrelated layers as in the benchmark.
+    _sampled_stack(dsa, oracle_mod, pattern, 200000, 62,
+                   rows=[1, 2048, 99999, 199999], att_rows=[1, 2048, 199999],
+                   corr=False, shared_q=True)

@@ -14,11 +14,22 @@ from gpu_util import to_dev_bf16
 pytestmark = pytest.mark.gpu
 
 ATOL, RTOL = 2e-2, 1e-2
-# MLA log-sum-exp: each CTA of a pair adds the peer's half of every score as
-# fp16 (relative rounding <= 2^-11), so a logit moves by at most
-# scale * 2^-11 * |partial score|; with 576-wide N(0, 0.5^2) rows the partial
-# scores stay below ~40, giving |dLSE| <= 1/24 * 2^-11 * 40 ~ 1e-3.
-LSE_ATOL = 1e-3
+# MLA log-sum-exp: the two CTAs of a pair each sum their half of every score
+# in fp32 and add the peer's fp32 partial, so a logit carries the error of an
+# fp32 sum of exact bf16 products, |de| <= scale * (D_qk + 2) * 2^-24 *
+# sum_c |q_c k_c| (recursive summation bound), and the softmax denominator the
+# rounding of k positive fp32 terms, relative k * 2^-24.  The bound below adds
+# both; LSE_ATOL covers the N(0, 0.5^2) rows of most tests (sum_c |q_c k_c| <
+# 250 there, so the dot term is < 1/24 * 578 * 2^-24 * 250 = 3.6e-4).
+LSE_ATOL = 1e-5 + 2048 * 2.0 ** -24 + 3.6e-4
+
+
+def _lse_bound(q_row, kv_rows, sel, scale):
+    """Per-head LSE error bound for one row (see LSE_ATOL) from its inputs."""
+    qf = synth.bf16_bits_to_f32(q_row).astype(np.float64)
+    kf = synth.bf16_bits_to_f32(kv_rows[sel[sel >= 0]]).astype(np.float64)
+    mag = (np.abs(qf) @ np.abs(kf).T).max(axis=1)          # [n_h]
+    return 1e-5 + len(kf) * 2.0 ** -24 + scale * (qf.shape[1] + 2) * 2.0 ** -24 * mag
 
 
 @pytest.fixture(scope="module")
@@ -274,3 +285,90 @@ def test_mla_prefill_200k_layer_sampled(dsa, oracle_mod):
         krows = synth.rows(seed, synth.KV, synth.NORMAL, layer, (B, L, 576), sel[i][:n].astype(np.uint64), sigma=0.5)
         o, _ = oracle_mod.sparse_attn_row(qrow, krows, krows, np.arange(n, dtype=np.int32), scale, Dv=512)
         _close(out[0, i].float().cpu().numpy(), o)
+
+
+def _int_rows(seed, shape, lo, hi):
+    """Integer-valued bf16 bit patterns uniform in [lo, hi] (exact in bf16)."""
+    rng = np.random.default_rng(seed)
+    return synth.f32_to_bf16_bits(rng.integers(lo, hi + 1, size=shape).astype(np.float32))
+
+
+def test_mla_large_partial_scores(dsa, oracle_mod):
+    # Integer query and latent rows in [16, 24]: every score is an exact fp32
+    # integer near 576 * 400 (each CTA's 256- or 320-column partial alone is
+    # far beyond the fp16 range), logits are ~9,600 apart from each other by
+    # whole multiples of 1/24, so the softmax is sharp and near-ties occur.
+    # The output must still agree with the fp64 oracle: nothing in the kernel
+    # saturates or loses the partial sums' precision.
+    B, L, k = 1, 600, 256
+    q = _int_rows(31, (B, L, 128, 576), 16, 24)
+    kv = _int_rows(32, (B, L, 576), 16, 24)
+    rng = np.random.default_rng(33)
+    idx = _random_rows(rng, B, L, 0, k)
+    scale = 1 / math.sqrt(576)
+    got, lse = _run_mla(dsa, q, kv, idx, 0, scale)
+    for i in [1, 2, 63, 64, 255, 256, 257, 411, 599]:
+        o, l = oracle_mod.sparse_attn_row(q[0, i], kv[0], kv[0], idx[0, i], scale, Dv=512)
+        _close(got[0, i], o)
+        bound = _lse_bound(q[0, i], kv[0], idx[0, i], scale)
+        assert np.all(np.abs(lse[0, i] - l) <= bound + 1e-6 * np.abs(l)), np.abs(lse[0, i] - l).max()
+
+
+def test_mla_wide_normal_inputs(dsa, oracle_mod):
+    # q and latent rows NORMAL(sigma = 8): logits spread over hundreds of
+    # units (a sharp softmax), partial scores in the thousands.
+    B, L, k = 1, 700, 512
+    q = synth.tensor(41, synth.Q, synth.NORMAL, 0, (B, L, 128, 576), sigma=8.0)
+    kv = synth.tensor(41, synth.KV, synth.NORMAL, 0, (B, L, 576), sigma=8.0)
+    rng = np.random.default_rng(43)
+    idx = _random_rows(rng, B, L, 0, k)
+    scale = 1 / math.sqrt(576)
+    got, lse = _run_mla(dsa, q, kv, idx, 0, scale)
+    for i in [1, 5, 64, 511, 512, 513, 699]:
+        o, l = oracle_mod.sparse_attn_row(q[0, i], kv[0], kv[0], idx[0, i], scale, Dv=512)
+        _close(got[0, i], o)
+        bound = _lse_bound(q[0, i], kv[0], idx[0, i], scale)
+        assert np.all(np.abs(lse[0, i] - l) <= bound + 1e-6 * np.abs(l)), np.abs(lse[0, i] - l).max()
+
+
+@pytest.mark.parametrize("mla", [False, True])
+def test_out_of_range_entries_are_skipped(dsa, oracle_mod, mla):
+    # Index entries at or beyond Lk (outside the sequence's rows) are skipped
+    # like -1 padding by both attention kernels: the output equals the
+    # oracle's over the remaining entries, and nothing outside the K/V rows
+    # of the sequence is read.
+    import torch
+    B, L, k = 2, 300, 64
+    rng = np.random.default_rng(51)
+    idx = _random_rows(rng, B, L, 0, k)
+    bad = idx.copy()
+    for b in range(B):
+        for i in range(3, L, 7):
+            n = min(i, k)
+            pos = rng.choice(n, size=max(1, n // 4), replace=False)
+            bad[b, i, pos] = L + rng.integers(0, 1 << 20, size=len(pos))
+    clean = np.where(bad >= L, -1, bad).astype(np.int32)
+    if mla:
+        q, kv = _mla_inputs(52, B, L, L)
+        scale = 1 / math.sqrt(576)
+        got, lse = _run_mla(dsa, q, kv, bad, 0, scale)
+        K = V = kv
+        Dv = 512
+    else:
+        n_h, D = 4, 64
+        q = synth.tensor(53, synth.Q, synth.NORMAL, 0, (B, L, n_h, D))
+        K = synth.tensor(53, synth.K_SEP, synth.NORMAL, 0, (B, L, D))
+        V = synth.tensor(53, synth.V_SEP, synth.NORMAL, 0, (B, L, D))
+        scale = 1 / math.sqrt(D)
+        lse_t = torch.empty((B, L, n_h), dtype=torch.float32, device="cuda")
+        out = dsa.sparse_attn(to_dev_bf16(q), to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(bad).cuda(),
+                              scale, D_v=D, lse=lse_t)
+        dsa.check_device_errors()
+        got, lse = out.float().cpu().numpy(), lse_t.cpu().numpy()
+        Dv = D
+    for b in range(B):
+        for i in (3, 10, 66, 101, 297):
+            o, l = oracle_mod.sparse_attn_row(q[b, i], K[b], V[b], clean[b, i], scale, Dv=Dv)
+            _close(got[b, i], o)
+            fin = np.isfinite(l)
+            np.testing.assert_allclose(lse[b, i][fin], l[fin], rtol=1e-4, atol=LSE_ATOL)

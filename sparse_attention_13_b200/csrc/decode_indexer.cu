@@ -165,7 +165,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint32_t* out = p.keys + static_cast<size_t>(b) * p.row_stride;
     for (int t = 0; t < n_tiles; ++t) {
       const int buf = t % kDecBufs;
-      if (!mbar_wait(&t_full[buf], (t / kDecBufs) & 1, abort_flag)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&t_full[buf], (t / kDecBufs) & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t v[H];
       if constexpr (H >= 32) {

@@ -474,7 +474,7 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int h = 0; h < 2; ++h) {
           if (it.nq[h] == 0) continue;
           const uint32_t buf = unit & 1;
-          if (!mbar_wait(&tmem_full[buf], (unit >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[buf], (unit >> 1) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
           float acc[kQPT];
           const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + buf * 256;

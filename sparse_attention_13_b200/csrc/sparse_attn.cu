@@ -520,7 +520,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const int stage = g % kStages;
         const int sb = g & 1;
         float s[32];
-        if (ok) ok = mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag));
         tc_fence_after();
         if (ok) {
           uint32_t v[32];
@@ -568,11 +568,15 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         ok = named_bar_and(pair_bar, 64, ok);
         if (!ok) break;
         const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]) * p.scale_log2;
-        if (cmax > m_run + kRescaleThresh) {
-          const float factor = ex2_approx(m_run - cmax);  // 0 when m_run = -inf
+        // Heads rescale independently, but the TMEM accesses below are
+        // warp-collective (.sync.aligned): the warp enters together when any
+        // of its heads needs it, and the others scale by exactly 1.
+        const bool grow = cmax > m_run + kRescaleThresh;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float factor = grow ? ex2_approx(m_run - cmax) : 1.f;  // 0 when m_run = -inf
           if (c > 0) {
             // O holds PV of the earlier chunks: wait for PV(g-1), scale my 128 columns
-            ok = mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag));
             tc_fence_after();
             if (ok) {
 #pragma unroll 1
@@ -588,8 +592,10 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
               tmem_st_wait();
             }
           }
-          l_run *= factor;
-          m_run = cmax;
+          if (grow) {
+            l_run *= factor;
+            m_run = cmax;
+          }
         }
         uint32_t pk[16];
         float e4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (short chains)
@@ -605,7 +611,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         l_run += (e4[0] + e4[1]) + (e4[2] + e4[3]);
         // P(g) overwrites the first 32 columns of S[g & 1] once the sender has
         // read them (both halves of this head read theirs before the pair barrier)
-        if (ok) ok = mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag));
         tc_fence_after();
         if (ok) {
           tmem_st32x16(t_lane + kSCol + sb * 64 + hf * 16, pk);
@@ -627,7 +633,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       const float l_lse_tot = l_tot;
       named_bar_sync(pair_bar + 4, 64);  // lsum is rewritten by the next item
       // epilogue: O / l
-      ok = mbar_wait(&bb->o_full, it_n & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bb->o_full, it_n & 1, abort_flag));
       tc_fence_after();
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float lse_v = l_lse_tot > 0.f ? (m_run + __log2f(l_lse_tot)) * 0.6931471805599453f : -INFINITY;

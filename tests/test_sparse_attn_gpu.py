@@ -316,7 +316,12 @@ def test_mla_large_partial_scores(dsa, oracle_mod):
 
 def test_mla_wide_normal_inputs(dsa, oracle_mod):
     # q and latent rows NORMAL(sigma = 8): logits spread over hundreds of
-    # units (a sharp softmax), partial scores in the thousands.
+    # units (a sharp softmax), partial scores in the thousands.  The softmax
+    # weights enter the P.V tensor-core product as bf16 (V is bf16, and one
+    # UMMA takes one type), whose unit roundoff is 2^-8; with weights summing
+    # to one that moves output column c by at most 2^-8 max_r |V[r, c]|, which
+    # at sigma = 8 (|V| up to ~28) exceeds the fixed 2e-2 of the benchmark's
+    # sigma = 0.5 inputs (there the term is < 0.007).  The bound is added.
     B, L, k = 1, 700, 512
     q = synth.tensor(41, synth.Q, synth.NORMAL, 0, (B, L, 128, 576), sigma=8.0)
     kv = synth.tensor(41, synth.KV, synth.NORMAL, 0, (B, L, 576), sigma=8.0)
@@ -326,7 +331,10 @@ def test_mla_wide_normal_inputs(dsa, oracle_mod):
     got, lse = _run_mla(dsa, q, kv, idx, 0, scale)
     for i in [1, 5, 64, 511, 512, 513, 699]:
         o, l = oracle_mod.sparse_attn_row(q[0, i], kv[0], kv[0], idx[0, i], scale, Dv=512)
-        _close(got[0, i], o)
+        sel = idx[0, i][idx[0, i] >= 0]
+        vmax = np.abs(synth.bf16_bits_to_f32(kv[0, sel, :512]).astype(np.float64)).max(axis=0)
+        err = np.abs(got[0, i] - o)
+        assert np.all(err <= ATOL + RTOL * np.abs(o) + 2.0 ** -8 * vmax[None, :]), err.max()
         bound = _lse_bound(q[0, i], kv[0], idx[0, i], scale)
         assert np.all(np.abs(lse[0, i] - l) <= bound + 1e-6 * np.abs(l)), np.abs(lse[0, i] - l).max()
 

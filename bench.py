@@ -47,10 +47,12 @@ WORKLOAD = ("prefill: B=1, L=200000, 16 layers FSSS x4 (1/4 F), H_I=64 d_I=128 k
             "576/512; decode: B=8, ctx 200000, 48 layers 1/4 F")
 
 
-def config_of(world):
+def config_of(world, shard_mode="replicas"):
     """The `config` object of the JSON line (the same for both arms)."""
-    return {"workload": WORKLOAD, "global_batch": world, "seq_len": PREFILL["L"],
-            "parallelism": f"dp{world} (independent replicas)",
+    zig = shard_mode == "zigzag" and world > 1
+    return {"workload": WORKLOAD, "global_batch": 1 if zig else world, "seq_len": PREFILL["L"],
+            "parallelism": (f"one sequence, zig-zag query chunks over {world} ranks" if zig
+                            else f"dp{world} (independent replicas)"),
             "l2": "inputs larger than L2 (126 MB) every step; no flush"}
 
 
@@ -271,7 +273,7 @@ def run_dsa(args):
     import torch
     import torch.distributed as dist
 
-    from sparse_attention_13_b200 import dsa, synth
+    from sparse_attention_13_b200 import dsa, shard, synth
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -320,9 +322,20 @@ def run_dsa(args):
     dims = dsa.make_dims(B=1, Lq=L, Lk=L, start_pos=0, H_I=P["H_I"], d_I=P["d_I"], k=k,
                          n_h=P["n_h"], D_qk=P["D_qk"], D_v=P["D_v"], scale=scale,
                          k_row_stride=P["D_qk"], v_row_stride=P["D_qk"])
-    ws = torch.empty(dsa.indexcache_forward_workspace(dims), dtype=torch.uint8, device=dev)
+    # Query rows this rank computes: the whole sequence (independent
+    # replicas), or its two zig-zag chunks of the one sequence, each run as a
+    # chunked prefill (start_pos = the chunk's first row) over the full caches.
+    zig = args.shard == "zigzag" and world > 1
+    chunks = shard.zigzag_chunks(L, world, rank) if zig else [(0, L)]
+
+    def chunk_dims(s, n):
+        return dsa.make_dims(B=1, Lq=n, Lk=L, start_pos=s, H_I=P["H_I"], d_I=P["d_I"], k=k,
+                             n_h=P["n_h"], D_qk=P["D_qk"], D_v=P["D_v"], scale=scale,
+                             k_row_stride=P["D_qk"], v_row_stride=P["D_qk"])
+
+    ws = torch.empty(max(dsa.indexcache_forward_workspace(chunk_dims(s, n)) for s, n in chunks),
+                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    n_launch = [0]
 
     def step(events=None):
         for l, role in enumerate(pat):
@@ -330,13 +343,17 @@ def run_dsa(args):
                 if events is not None:
                     events["idx"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
                     events["idx"][-1][0].record(stream)
-                dsa.indexer_topk(q_idx[l], k_idx[l], w[l], k, out=idx, ws=ws)
+                for s, n in chunks:
+                    dsa.indexer_topk(q_idx[l][:, s:s + n], k_idx[l], w[l][:, s:s + n], k, start_pos=s,
+                                     out=idx[:, s:s + n], ws=ws)
                 if events is not None:
                     events["idx"][-1][1].record(stream)
             if events is not None:
                 events["attn"].append((torch.cuda.Event(True), torch.cuda.Event(True)))
                 events["attn"][-1][0].record(stream)
-            dsa.sparse_attn(q, kv[l], kv[l], idx, scale, D_v=P["D_v"], out=out, ws=ws)
+            for s, n in chunks:
+                dsa.sparse_attn(q[:, s:s + n], kv[l], kv[l], idx[:, s:s + n], scale, D_v=P["D_v"], start_pos=s,
+                                out=out[:, s:s + n], ws=ws)
             if events is not None:
                 events["attn"][-1][1].record(stream)
 
@@ -360,24 +377,26 @@ def run_dsa(args):
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["idx"])
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["attn"])
-    tokens = L * world
-    a_units = attn_units(L, 0, k)
-    i_pairs = indexer_pairs(L, 0)
+    # this rank's work per layer (its chunks; the whole sequence for replicas)
+    a_units = sum(shard.attention_rows(s, n, k) for s, n in chunks)
+    i_pairs = sum(shard.indexer_pairs(s, n) for s, n in chunks)
     attn_flops = a_units * 2 * P["n_h"] * (P["D_qk"] + P["D_v"])
     idx_flops = i_pairs * 2 * P["H_I"] * P["d_I"]
+    job_tokens = L if zig else L * world  # one sequence split, or one per rank
     result["prefill"] = dict(
-        ms_per_step=ms, tokens_per_s=job_rate(L, world, ms), idx_ms=idx_ms, attn_ms=attn_ms,
+        ms_per_step=ms, tokens_per_s=job_tokens / (ms / 1e3), idx_ms=idx_ms, attn_ms=attn_ms,
         indexer_share=nF * idx_ms / (nF * idx_ms + len(pat) * attn_ms),
         attn_tflops=attn_flops / attn_ms / 1e9, idx_tflops=idx_flops / idx_ms / 1e9,
-        attn_flops=attn_flops, idx_flops=idx_flops, clocks=clk,
-        launches=args.steps * (nF + len(pat)))
+        attn_flops=attn_flops, idx_flops=idx_flops, clocks=clk, chunks=chunks,
+        scaling="strong" if zig else "weak",
+        launches=args.steps * len(chunks) * (nF + len(pat)))
 
     # The ratio sweep of the long prefill (1/1 and 1/2 beside the 1/4 stack
     # timed above): the same 16 layers and shapes, with an indexer on every
     # layer, or on every other layer.  Extra F layers get their own indexer
     # inputs.  Kernels are warm; one warm-up step and a short timed region.
     sweep = {}
-    if not args.no_sweep:
+    if not args.no_sweep and not zig:
         extra = []
         for l in range(len(pat)):
             if l not in q_idx:
@@ -413,50 +432,95 @@ def run_dsa(args):
                 warmup=1 if ratio != P["ratio"] else args.warmup)
         for l in extra:
             del q_idx[l], k_idx[l], w[l]
+        del lin
         torch.cuda.empty_cache()
     result["prefill"]["sweep"] = sweep
 
-    # e2e through the public API with host buffers
+    # The low-precision selector ([IDX] §5.4) on the first F layer's inputs,
+    # timed per launch beside the bf16 indexer (the call quantises q_idx and
+    # k_idx into its workspace, included in the time).
+    lowprec = {}
+    if not args.no_sweep and not zig:
+        for fmt in ("e4m3", "e2m1"):
+            lws = torch.empty(dsa.indexer_topk_lowprec_workspace(1, L, L, 0, P["H_I"], P["d_I"], k, fmt),
+                              dtype=torch.uint8, device=dev)
+            run = lambda: dsa.indexer_topk_lowprec(q_idx[0], k_idx[0], w[0], k, fmt=fmt, out=idx, ws=lws)  # noqa: E731
+            run()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+            e0.record(stream)
+            for _ in range(2):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            lms = max_over_ranks(e0.elapsed_time(e1) / 2)
+            lowprec[fmt] = {"ms_per_launch": lms, "speedup_vs_bf16": idx_ms / lms,
+                            "tflops_equiv": idx_flops / lms / 1e9}
+            del lws
+        dsa.check_device_errors()
+    result["prefill"]["lowprec"] = lowprec
+
+    # e2e through the public API with host buffers: every step copies in the
+    # caches and this rank's query-side rows, and copies its output rows back
     host_in = []
     for l in sorted(q_idx):
-        host_in += [(q_idx[l], None), (k_idx[l], None), (w[l], None)]
-    host_in += [(t, None) for t in kv] + [(q, None)]
+        host_in += [(k_idx[l], None)] + [(q_idx[l][:, s:s + n], None) for s, n in chunks] + \
+                   [(w[l][:, s:s + n], None) for s, n in chunks]
+    host_in += [(t, None) for t in kv] + [(q[:, s:s + n], None) for s, n in chunks]
     host_in = [(d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True)) for d, _ in host_in]
     for d, h in host_in:
         h.copy_(d)
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    out_dev = [out[:, s:s + n] for s, n in chunks]
+    out_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out_dev]
     h2d = sum(d.numel() * d.element_size() for d, _ in host_in)
-    d2h = out.numel() * out.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in out_dev)
     # a second device set of every input and of the output (double buffering)
     set_dev = [[d for d, _ in host_in], [torch.empty_like(d) for d, _ in host_in]]
-    set_out = [out, torch.empty_like(out)]
+    set_out = [out_dev, [torch.empty_like(o) for o in out_dev]]
+    pos = {id(d): i for i, (d, _) in enumerate(host_in)}
 
-    def layers_of(b):
-        dmap = {id(d0): d1 for d0, d1 in zip(set_dev[0], set_dev[b])}
+    def layers_of(b, c):
+        # the layer list of chunk c on device set b
+        sel = lambda d: set_dev[b][pos[id(d)]]  # noqa: E731
         res = []
         for l, role in enumerate(pat):
-            L_ = dict(q=dmap[id(q)], kbuf=dmap[id(kv[l])], vbuf=dmap[id(kv[l])], out=set_out[b])
+            L_ = dict(q=sel(q_views[c]), kbuf=sel(kv[l]), vbuf=sel(kv[l]), out=set_out[b][c])
             if role == "F":
-                L_.update(q_idx=dmap[id(q_idx[l])], k_idx=dmap[id(k_idx[l])], w=dmap[id(w[l])])
+                L_.update(q_idx=sel(qi_views[l][c]), k_idx=sel(k_idx[l]), w=sel(w_views[l][c]))
             res.append(L_)
         return res
 
-    set_layers = [layers_of(0), layers_of(1)]
+    # the views registered in host_in, by chunk
+    q_views = [host_in[len(host_in) - len(chunks) + c][0] for c in range(len(chunks))]
+    qi_views, w_views = {}, {}
+    base = 0
+    for l in sorted(q_idx):
+        qi_views[l] = [host_in[base + 1 + c][0] for c in range(len(chunks))]
+        w_views[l] = [host_in[base + 1 + len(chunks) + c][0] for c in range(len(chunks))]
+        base += 1 + 2 * len(chunks)
+    set_layers = [[layers_of(b, c) for c in range(len(chunks))] for b in range(2)]
     h2d_pairs = [[(d, h) for d, (_, h) in zip(set_dev[b], host_in)] for b in range(2)]
-    d2h_pairs = [[(set_out[b], out_h)] for b in range(2)]
+    d2h_pairs = [[(set_out[b][c], out_h[c]) for c in range(len(chunks))] for b in range(2)]
+    cdims = [chunk_dims(s, n) for s, n in chunks]
+    cidx = [idx[:, s:s + n] for s, n in chunks]
 
     def e2e_forward(b):
-        dsa.indexcache_forward(pat, set_layers[b], dims, idx, ws=ws)
+        for c in range(len(chunks)):
+            dsa.indexcache_forward(pat, set_layers[b][c], cdims[c], cidx[c], ws=ws)
 
     pipelined_e2e(torch, dev, stream, h2d_pairs, e2e_forward, d2h_pairs, args.warmup)
     barrier()
     e2e_ms = max_over_ranks(pipelined_e2e(torch, dev, stream, h2d_pairs, e2e_forward, d2h_pairs, args.steps))
     barrier()
     dsa.check_device_errors()
-    result["prefill"]["e2e"] = {"value": job_rate(L, world, e2e_ms), "unit": "tokens/s",
+    result["prefill"]["e2e"] = {"value": job_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del host_in, out_h, q_idx, k_idx, w, kv, q, out, idx, ws, set_dev, set_out, set_layers, h2d_pairs, d2h_pairs
+    del out_dev, q_views, qi_views, w_views, cidx, pos
+    d = h = t = None  # loop variables above still name device tensors
+    torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
+    assert torch.cuda.memory_allocated(dev) < (1 << 30), "prefill buffers still referenced"
 
     # ---------------------------------------------------------------- decode
     D = dict(DECODE)
@@ -852,7 +916,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": config_of(args.gpus),
+            "config": config_of(args.gpus, args.shard),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count() or 1,
                              "kind": "oracle",
                              "sample": f"per step: 1 indexer row at t = L/2 (the mean causal row) and "
@@ -938,6 +1002,51 @@ def kernel_case(name, seq, reps):
     torch.cuda.synchronize()
     dsa.check_device_errors()
     print(f"{name} seq={seq}: {e0.elapsed_time(e1) / reps:.3f} ms/launch", flush=True)
+
+
+def lowprec_case(seq, kk=2048, reps=2):
+    """The low-precision selector ([IDX] §5.4) against the exact one on
+    normal inputs (B = 1, L = seq, 64 indexer heads x 128, k = kk): Recall@k
+    of each format's selection over the rows t >= k, and CUDA-event times of
+    the bf16 indexer and of both formats.  Prints one JSON line."""
+    import torch
+
+    from sparse_attention_13_b200 import dsa, synth
+    dev = torch.device("cuda", 0)
+    L = seq
+    q = torch.empty((1, L, 64, 128), dtype=torch.bfloat16, device=dev)
+    kt = torch.empty((1, L, 128), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((1, L, 64), dtype=torch.float32, device=dev)
+    synth.fill_cuda(q, SEED, synth.Q_IDX, synth.NORMAL, 0, sigma=1.0)
+    synth.fill_cuda(kt, SEED, synth.K_IDX, synth.NORMAL, 0, sigma=1.0)
+    synth.fill_cuda(w, SEED, synth.W, synth.NORMAL, 0, sigma=1.0)
+    w = w.abs() / 64.0  # positive head weights (the softmax-normalised gates of the pages' indexer)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        for _ in range(reps):
+            r = fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return r, e0.elapsed_time(e1) / reps
+
+    ws = torch.empty(dsa.indexer_topk_workspace(1, L, L, 0, 64, 128, kk), dtype=torch.uint8, device=dev)
+    exact, t_exact = timed(lambda: dsa.indexer_topk(q, kt, w, kk, ws=ws))
+    exact = exact.clone()
+    res = {"tool": "lowprec_selector", "workload": f"B=1, L={L}, H_I=64, d_I=128, k={kk}, normal q/k (sigma 1), "
+           "positive head weights", "data": "synthetic", "bf16_ms": t_exact}
+    for fmt in ("e4m3", "e2m1"):
+        lws = torch.empty(dsa.indexer_topk_lowprec_workspace(1, L, L, 0, 64, 128, kk, fmt), dtype=torch.uint8,
+                          device=dev)
+        sel, t = timed(lambda: dsa.indexer_topk_lowprec(q, kt, w, kk, fmt=fmt, ws=lws))
+        inter = dsa.index_overlap(exact[:, kk:].contiguous(), sel[:, kk:].contiguous())
+        res[fmt] = {"ms": t, "speedup_vs_bf16": t_exact / t,
+                    "recall_at_k": float(inter.float().mean()) / kk}
+    dsa.check_device_errors()
+    print(json.dumps(res), flush=True)
 
 
 def csa_layer(seq, kk=512, m=4, reps=2):
@@ -1090,15 +1199,22 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default="",
                     help="profiling: indexer|attn|decode_idx|decode_attn|decode_step; "
-                         "quality runs the selection-quality tools, csa one CSA-style layer")
+                         "quality runs the selection-quality tools, csa one CSA-style layer, "
+                         "lowprec the low-precision selector's recall and times")
     ap.add_argument("--reps", type=int, default=2)
     ap.add_argument("--decode-steps", type=int, default=2000,
                     help="CUDA-graph replays in the decode timed region")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "zigzag"],
+                    help="N > 1: independent replicas (weak scaling) or one sequence split into zig-zag "
+                         "query chunks across the ranks (strong scaling)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the ratio sweep and the config-2/config-3 lines (short runs)")
     args = ap.parse_args()
     if args.kernel_case == "quality":
         selection_quality(args.seq or 8192)
+        return
+    if args.kernel_case == "lowprec":
+        lowprec_case(args.seq or 65536, reps=args.reps)
         return
     if args.kernel_case == "csa":
         csa_layer(args.seq or 200000, reps=args.reps)
@@ -1122,9 +1238,9 @@ def main():
     line = {
         "metric": METRIC, "value": pf["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_per_step"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": pf["scaling"], "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(world),
+        "config": config_of(world, args.shard),
         "roofline": {"bound": "tensor", "kernel": "mla_sparse_attn", "achieved": pf["attn_tflops"],
                      "peak": tc_peak, "unit": "TFLOP/s", "frac": pf["attn_tflops"] / tc_peak,
                      "traffic": attn_tr, "peak_kind": f"{peak_kind} bf16 sustained",
@@ -1134,6 +1250,9 @@ def main():
                              "traffic": idx_tr, "per_launch_flops": pf["idx_flops"],
                              "avg_launch_ms": pf["idx_ms"]},
         "indexer_share": pf["indexer_share"],
+        "lowprec": {"workload": "one F layer of the prefill (L=200000, 64 x 128, k=2048), MX operands "
+                                "quantised inside the call, bf16 scores; 1 warm-up + 2 launches",
+                    "bf16_ms_per_launch": pf["idx_ms"], "formats": pf["lowprec"]},
         "sweep": {"workload": "prefill B=1, L=200000, 16 layers, F ratios 1/1 (F x16), 1/2 (FS x8), "
                               "1/4 (FSSS x4); indexer_ms_expected = M/N x the all-F indexer time per step",
                   "ratios": pf["sweep"]},
@@ -1162,7 +1281,7 @@ def main():
                                 "decode_ms_per_step": cb["decode_ms_per_step"],
                                 "decode_sample": cb["decode_sample"]}
         if host_cores > 1:
-            line["cpu_baseline"]["row_parallel"] = oracle_parallel_sample(min(host_cores, 64))
+            line["cpu_baseline"]["row_parallel"] = oracle_parallel_sample(min(host_cores, 16))
     print(json.dumps(line), flush=True)
 
 

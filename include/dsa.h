@@ -151,6 +151,107 @@ dsa_status indexcache_forward(const char *pattern, int n_layers,
                               void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Variable-length batches.  [IDX] §4.3 (the cost account of DSA, with its
+ * note that prefill and decode requests are served differently): a serving
+ * batch mixes sequences of different lengths and positions.  The pages
+ * describe one sequence at a time; a batch is the same computation applied
+ * to each sequence independently.  Rows of all sequences are packed:
+ *   query-side tensors (q_idx, w, q, out, lse, idx) hold the rows of
+ *   sequence b at rows cu_q[b] .. cu_q[b+1]-1, in order; row i of sequence b
+ *   sits at absolute position t = start_pos[b] + i and sees s < t;
+ *   key-side tensors (k_idx, the K/V or latent rows) hold sequence b's
+ *   cached positions s = 0 .. at rows cu_k[b] + s, s < cu_k[b+1] - cu_k[b].
+ * The three arrays are DEVICE int32 arrays the caller owns; the host values
+ * total_q = cu_q[B], total_k = cu_k[B] and the bounds max_Lq >= every
+ * cu_q[b+1]-cu_q[b] and max_Lk >= every cu_k[b+1]-cu_k[b] size the launch.
+ * Contract, checked on the device by dsa_check_varlen (the host cannot read
+ * the arrays without synchronising): cu_q and cu_k start at 0, never
+ * decrease and end at total_q / total_k; start_pos[b] >= 0; start_pos[b] +
+ * (cu_q[b+1]-cu_q[b]) - 1 <= cu_k[b+1]-cu_k[b]; the per-sequence lengths
+ * respect the bounds.  A batch breaking it gets unspecified rows but no
+ * access outside the tensors.  Sequences with no query rows are allowed.
+ * When every sequence has exactly one query row (max_Lq = 1, total_q = B:
+ * decode), the indexer takes the streaming decode kernels. */
+typedef struct {
+  int B;                    /* sequences */
+  const int32_t *cu_q;      /* device [B + 1] query-row offsets */
+  const int32_t *cu_k;      /* device [B + 1] cached-row offsets */
+  const int32_t *start_pos; /* device [B] position of each sequence's first row */
+  int total_q, total_k;     /* cu_q[B], cu_k[B] */
+  int max_Lq, max_Lk;       /* bounds of the per-sequence lengths */
+} dsa_varlen;
+
+/* dsa_indexer_topk over a variable-length batch: q_idx [total_q, H_I, d_I],
+ * k_idx [total_k, d_I], w [total_q, H_I], idx [total_q, k] (written), with
+ * the semantics, limits and row form of dsa_indexer_topk per sequence. */
+size_t dsa_indexer_topk_varlen_workspace(const dsa_varlen *vl, int H_I, int d_I, int k);
+dsa_status dsa_indexer_topk_varlen(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
+                                   const float *w, const dsa_varlen *vl, int H_I,
+                                   int d_I, int k, int32_t *idx, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* dsa_sparse_attn over a variable-length batch: q [total_q, n_h, D_qk],
+ * K/V rows kbuf + r * k_row_stride for r < total_k (sequence b's position s
+ * at r = cu_k[b] + s), idx [total_q, k], out [total_q, n_h, D_v], lse
+ * [total_q, n_h] (may be NULL).  Index entries outside [0, the sequence's
+ * cache length) are skipped. */
+size_t dsa_sparse_attn_varlen_workspace(const dsa_varlen *vl, int n_h, int D_v, int k);
+dsa_status dsa_sparse_attn_varlen(const dsa_bf16 *q, const dsa_bf16 *kbuf,
+                                  int64_t k_row_stride, const dsa_bf16 *vbuf,
+                                  int64_t v_row_stride, const int32_t *idx,
+                                  const dsa_varlen *vl, int n_h, int D_qk, int D_v,
+                                  int k, float scale, dsa_bf16 *out, float *lse,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* indexcache_forward over a variable-length batch: the layer loop above with
+ * packed per-layer tensors.  dims supplies H_I, d_I, k, n_h, D_qk, D_v, scale
+ * and the row strides; its B, Lq, Lk and start_pos are ignored (vl gives
+ * them).  idx_cache is [total_q, k]. */
+size_t indexcache_forward_varlen_workspace(const dsa_dims *dims, const dsa_varlen *vl);
+dsa_status indexcache_forward_varlen(const char *pattern, int n_layers,
+                                     const dsa_layer_io *layers, const dsa_dims *dims,
+                                     const dsa_varlen *vl, int32_t *idx_cache, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/* Checks the contract of a variable-length batch on the device and writes
+ * the number of sequences that break it to *bad_seqs (one device int,
+ * overwritten; read it after the stream completes).  Allocates nothing. */
+dsa_status dsa_check_varlen(const dsa_varlen *vl, int *bad_seqs, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Low-precision selector.  [IDX] §5.4: the indexer's QK product on FP4 (or
+ * FP8) operands and the index score quantised from FP32 to BF16 before the
+ * top-k, trading exactness of the selection for speed.  The pages name the
+ * formats only; the element and scale rules here are those of the OCP
+ * Microscaling (MX) v1.0 format that block-scaled tensor-core products use:
+ * along d_I, every 32 consecutive elements of a row share the power-of-two
+ * scale X = 2^(floor(log2 amax) - emax) (emax = 8 for E4M3, 2 for E2M1),
+ * held as an 8-bit exponent; each element becomes the format value nearest
+ * to x / X (ties to even, saturating).  Then, per query row t,
+ *   I[t,s] = bf16( sum_j w[t,j] * ReLU(q~[t,j,:] . k~[s,:]) )
+ * over s < t (q~, k~ the dequantised values; the head dots are fp32 sums of
+ * exact products), and S_t = TopK_k with the tie rule and row form of
+ * dsa_indexer_topk.  Inputs, output and row conventions are those of
+ * dsa_indexer_topk; the call quantises q_idx and k_idx into the workspace.
+ * Supported: H_I = 64, d_I = 128, k <= 2048, fmt DSA_FMT_E4M3 or
+ * DSA_FMT_E2M1.  Integer inputs in [-4, 4] quantise without loss. */
+#define DSA_FMT_E4M3 0
+#define DSA_FMT_E2M1 1
+size_t dsa_indexer_topk_lowprec_workspace(int B, int Lq, int Lk, int start_pos, int H_I,
+                                          int d_I, int k, int fmt);
+dsa_status dsa_indexer_topk_lowprec(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx,
+                                    const float *w, int B, int Lq, int Lk, int start_pos,
+                                    int H_I, int d_I, int k, int fmt, int32_t *idx, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/* MX quantisation of bf16 rows (the rule above): x [rows, cols] bf16 ->
+ * codes [rows, cols] (one byte per element: an E4M3 code, or an E2M1 code in
+ * bits 2..5 of its byte) and scales [rows, cols / 32] (the block exponent E
+ * as E + 127).  Supported: cols = 128. */
+dsa_status dsa_mx_quantize(const dsa_bf16 *x, int64_t rows, int cols, int fmt,
+                           uint8_t *codes, uint8_t *scales, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Allocation-free variant of dsa_indexer_topk.  The pages describe no such
  * entry point; it exists for callers that cannot provide device memory on
  * demand -- an engine whose allocator already owns all of HBM, a C program

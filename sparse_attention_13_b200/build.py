@@ -19,7 +19,7 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-s
 
 LIBS = {
     "libdsa.so": ["dsa_api.cu", "indexer_topk.cu", "decode_indexer.cu", "sparse_attn.cu", "noalloc.cu",
-                  "selection_quality.cu", "csa.cu"],
+                  "selection_quality.cu", "csa.cu", "lowprec.cu"],
     "libdsa_synth.so": ["synth.cu"],
 }
 DEPS = ["dsa_ptx.cuh", "dsa_internal.h"]

@@ -67,6 +67,11 @@ struct DecParams {
   uint32_t* keys;        // [B][row_stride] score keys
   int* hist;             // [B][n_split][4096] per-CTA key histograms
   unsigned int* err;
+  // Variable-length batches (both null for a uniform batch): sequence b's
+  // row sits at t = sp[b] (at most T) and its keys are rows cu_k[b] ... of
+  // the packed key tensor.
+  const int* sp;
+  const int* cu_k;
   int B, row_stride, T, n_split, split_len;
 };
 
@@ -94,8 +99,6 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int b = blockIdx.x / p.n_split;
   const int sp = blockIdx.x % p.n_split;
   const int s_begin = sp * p.split_len;
-  const int s_end = min(p.T, s_begin + p.split_len);
-  const int n_tiles = s_end > s_begin ? (s_end - s_begin + kTile - 1) / kTile : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) { mbar_init(&key_full[s], 1); mbar_init(&key_empty[s], 1); }
@@ -115,6 +118,13 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
   pdl_wait();
+  // the row's visible keys (per sequence when varlen; read after the wait,
+  // since earlier work in the stream may write the positions)
+  const int T = p.sp ? min(max(__ldg(p.sp + b), 0), p.T) : p.T;
+  const int k_row0 = p.cu_k ? __ldg(p.cu_k + b) : 0;
+  const int tb = p.cu_k ? 0 : b;
+  const int s_end = min(T, s_begin + p.split_len);
+  const int n_tiles = s_end > s_begin ? (s_end - s_begin + kTile - 1) / kTile : 0;
 
   if (warp == kDecTmaWarp) {
     if (lane == 0 && n_tiles > 0) {
@@ -129,7 +139,7 @@ decode_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_arrive_expect_tx(&key_full[stage], C::kStageBytes);
         uint8_t* dst = key_smem + stage * C::kStageBytes;
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kKeyChunkBytes, &tm_k, &key_full[stage], c * 64, s_begin + t * kTile, b);
+          tma_load_3d(dst + c * C::kKeyChunkBytes, &tm_k, &key_full[stage], c * 64, k_row0 + s_begin + t * kTile, tb);
       }
     }
   } else if (warp == kDecMmaWarp) {
@@ -288,7 +298,8 @@ __device__ __forceinline__ void pick_bin(int c, int bin, int kk, int base_above,
 //              passes over the slices with cluster-summed histograms.
 __global__ void __cluster_dims__(kClusterRanks, 1, 1) __launch_bounds__(kTopkThreads, 1)
 decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hist, int n_split,
-                   int32_t* __restrict__ idx, int row_stride, int T, int k, unsigned int* err) {
+                   int32_t* __restrict__ idx, int row_stride, int T_max, const int* __restrict__ Ts, int k,
+                   unsigned int* err) {
   extern __shared__ __align__(128) uint8_t topk_smem[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
   uint32_t* slice = reinterpret_cast<uint32_t*>(topk_smem + kTopkSharedBytes);
@@ -296,10 +307,6 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   const unsigned lt_mask = (1u << lane) - 1u;
   const int rank = static_cast<int>(cluster_ctarank());
   const size_t row = blockIdx.x / kClusterRanks;
-  const int per = round_up((T + kClusterRanks - 1) / kClusterRanks, 4);
-  const int lo = min(T, rank * per);
-  const int n = min(T, lo + per) - lo;
-  const int nw = (n + 31) / 32;
 
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
@@ -309,6 +316,13 @@ decode_topk_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ hi
   __syncthreads();
   pdl_trigger();
   pdl_wait();
+  // the row's visible keys: one count for a uniform batch, per sequence when
+  // varlen (uniform across the cluster: every CTA reads the same value)
+  const int T = Ts ? min(max(__ldg(Ts + row), 0), T_max) : T_max;
+  const int per = round_up((T + kClusterRanks - 1) / kClusterRanks, 4);
+  const int lo = min(T, rank * per);
+  const int n = min(T, lo + per) - lo;
+  const int nw = (n + 31) / 32;
   if (tid == 0 && n > 0) {
     const uint32_t bytes = static_cast<uint32_t>(round_up(n, 4)) * 4u;
     mbar_arrive_expect_tx(&sh.bar, bytes);
@@ -650,8 +664,10 @@ size_t decode_indexer_ws_bytes(int B, int Lk) {
 
 dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w, int B,
                                  int Lk, int start_pos, int H, int d, int k, int32_t* idx, void* ws,
-                                 size_t ws_bytes, cudaStream_t stream) {
-  const int T = start_pos;
+                                 size_t ws_bytes, cudaStream_t stream, const DecodeVarlen* vl) {
+  // uniform: every row at t = start_pos; varlen: row b at t = sp[b] <= Lk
+  // (the batch's longest cache) over the packed keys
+  const int T = vl ? Lk : start_pos;
   if (ws_bytes < decode_indexer_ws_bytes(B, Lk)) return set_error(DSA_ERR_WORKSPACE, "indexer workspace too small");
   const int sms = device_sm_count();
   if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
@@ -663,13 +679,17 @@ dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, c
   p.hist = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + keys_bytes(B, Lk));
   p.err = device_error_word();
   if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+  p.sp = vl ? vl->sp : nullptr;
+  p.cu_k = vl ? vl->cu_k : nullptr;
   p.B = B; p.row_stride = round_up(Lk, 4); p.T = T; p.n_split = n_split;
   p.split_len = ((tiles + n_split - 1) / n_split) * kTile;
   CUtensorMap tq, tk;
   if (!encode_tiled_3d(&tq, q_idx, d, H, B, static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(H) * d * 2,
                        64, H, CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(DSA_ERR_CUDA, "tensor map for q_idx failed");
-  if (!encode_tiled_3d(&tk, k_idx, d, Lk, B, static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(Lk) * d * 2,
+  const uint64_t krows = vl ? static_cast<uint64_t>(vl->total_k) : static_cast<uint64_t>(Lk);
+  const uint64_t kbatch = vl ? 1u : static_cast<uint64_t>(B);
+  if (!encode_tiled_3d(&tk, k_idx, d, krows, kbatch, static_cast<uint64_t>(d) * 2, krows * d * 2,
                        64, kTile, CU_TENSOR_MAP_SWIZZLE_128B))
     return set_error(DSA_ERR_CUDA, "tensor map for k_idx failed");
   const int grid = B * n_split;
@@ -687,7 +707,7 @@ dsa_status decode_indexer_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, c
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k smem attribute: ") + cudaGetErrorString(e));
   e = launch_pdl(decode_topk_kernel, dim3(B * kClusterRanks), dim3(kTopkThreads), tsmem, stream,
                  static_cast<const uint32_t*>(p.keys), static_cast<const int*>(p.hist), n_split, idx,
-                 p.row_stride, T, k, p.err);
+                 p.row_stride, T, p.sp, k, p.err);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("decode top-k launch: ") + cudaGetErrorString(e));
   return DSA_OK;

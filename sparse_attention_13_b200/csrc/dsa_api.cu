@@ -50,14 +50,14 @@ dsa_status set_error(dsa_status st, const std::string& msg) {
 
 bool encode_tiled_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                      uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
-                     CUtensorMapSwizzle swizzle) {
+                     CUtensorMapSwizzle swizzle, CUtensorMapDataType dtype) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
   const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -170,6 +170,22 @@ __global__ void full_visible_rows_kernel(int32_t* __restrict__ idx, int64_t n, i
   }
 }
 
+// Contract of a variable-length batch (include/dsa.h), one thread per
+// sequence: offsets start at 0, never decrease, end at the totals; lengths
+// within the bounds; every query row within its cache (t <= Lk_b).
+__global__ void check_varlen_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k,
+                                    const int* __restrict__ sp, int B, int total_q, int total_k, int max_Lq,
+                                    int max_Lk, int* bad) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
+    const int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_k[b], k1 = cu_k[b + 1];
+    bool ok = q1 >= q0 && k1 >= k0 && q1 - q0 <= max_Lq && k1 - k0 <= max_Lk && sp[b] >= 0 &&
+              static_cast<long long>(sp[b]) + (q1 - q0) - 1 <= static_cast<long long>(k1 - k0);
+    if (b == 0) ok = ok && q0 == 0 && k0 == 0;
+    if (b == B - 1) ok = ok && q1 == total_q && k1 == total_k;
+    if (!ok) atomicAdd(bad, 1);
+  }
+}
+
 }  // namespace dsa
 
 using namespace dsa;
@@ -192,6 +208,21 @@ dsa_status check_indexer_args(const dsa_bf16* q_idx, const dsa_bf16* k_idx, cons
                      "dsa_indexer_topk: need H_I in {4,8,16,32,64}, d_I in {32,64,128}, k <= 2048");
   if (static_cast<long long>(Lq) * H > (1ll << 31) - 1 || static_cast<long long>(B) * Lq * k > (1ll << 40))
     return set_error(DSA_ERR_UNSUPPORTED, "dsa_indexer_topk: tensor too large");
+  return DSA_OK;
+}
+
+dsa_status check_varlen_host(const dsa_varlen* vl, VarlenArgs* out) {
+  if (!vl) return set_error(DSA_ERR_INVALID_ARG, "varlen: null batch descriptor");
+  if (!vl->cu_q || !vl->cu_k || !vl->start_pos)
+    return set_error(DSA_ERR_INVALID_ARG, "varlen: null offset or position array");
+  if ((reinterpret_cast<uintptr_t>(vl->cu_q) | reinterpret_cast<uintptr_t>(vl->cu_k) |
+       reinterpret_cast<uintptr_t>(vl->start_pos)) & 3u)
+    return set_error(DSA_ERR_INVALID_ARG, "varlen: offset arrays must be 4-byte aligned");
+  if (vl->B < 1 || vl->total_q < 1 || vl->total_k < 1 || vl->max_Lq < 1 || vl->max_Lk < 1)
+    return set_error(DSA_ERR_INVALID_ARG, "varlen: sizes must be positive");
+  if (vl->max_Lq > vl->total_q || vl->max_Lk > vl->total_k)
+    return set_error(DSA_ERR_INVALID_ARG, "varlen: a per-sequence bound exceeds the total");
+  if (out) *out = VarlenArgs{vl->cu_q, vl->cu_k, vl->start_pos, vl->total_q, vl->total_k};
   return DSA_OK;
 }
 
@@ -306,6 +337,119 @@ dsa_status indexcache_forward(const char* pattern, int n_layers, const dsa_layer
                                     d.scale, L.out, L.lse, ws, ws_bytes, stream);
     if (st != DSA_OK) return st;
   }
+  return DSA_OK;
+}
+
+size_t dsa_indexer_topk_varlen_workspace(const dsa_varlen* vl, int H_I, int d_I, int k) {
+  if (check_varlen_host(vl, nullptr) != DSA_OK || k < 1) return 0;
+  return indexer_varlen_ws_bytes(vl->B, vl->max_Lq, vl->max_Lk, vl->total_q, H_I, d_I, k);
+}
+
+dsa_status dsa_indexer_topk_varlen(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
+                                   const dsa_varlen* vl, int H_I, int d_I, int k, int32_t* idx, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  VarlenArgs va{};
+  dsa_status st = check_varlen_host(vl, &va);
+  if (st != DSA_OK) return st;
+  // the per-sequence limits of dsa_indexer_topk, on the batch's bounds
+  st = check_indexer_args(q_idx, k_idx, w, 1, vl->max_Lq, vl->max_Lk, 0, H_I, d_I, k, idx);
+  if (st != DSA_OK) return st;
+  if (static_cast<long long>(vl->total_q) * H_I > (1ll << 31) - 1 ||
+      static_cast<long long>(vl->total_q) * k > (1ll << 40))
+    return set_error(DSA_ERR_UNSUPPORTED, "dsa_indexer_topk_varlen: tensor too large");
+  if (!ws || !aligned16(ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_indexer_topk_varlen: null or misaligned workspace");
+  if (ws_bytes < dsa_indexer_topk_varlen_workspace(vl, H_I, d_I, k))
+    return set_error(DSA_ERR_WORKSPACE, "dsa_indexer_topk_varlen: workspace too small");
+  st = indexer_topk_launch(q_idx, k_idx, w, vl->B, vl->max_Lq, vl->max_Lk, 0, H_I, d_I, k, idx, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream), &va);
+  if (st == DSA_OK) g_indexer_launches.fetch_add(1);
+  return st;
+}
+
+size_t dsa_sparse_attn_varlen_workspace(const dsa_varlen* vl, int n_h, int D_v, int k) {
+  if (check_varlen_host(vl, nullptr) != DSA_OK || n_h < 1 || D_v < 1 || k < 1) return 0;
+  return sparse_attn_ws_rows(vl->total_q, n_h, D_v, k);
+}
+
+dsa_status dsa_sparse_attn_varlen(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
+                                  const dsa_bf16* vbuf, int64_t v_row_stride, const int32_t* idx,
+                                  const dsa_varlen* vl, int n_h, int D_qk, int D_v, int k, float scale,
+                                  dsa_bf16* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  VarlenArgs va{};
+  dsa_status st = check_varlen_host(vl, &va);
+  if (st != DSA_OK) return st;
+  if (!q || !kbuf || !vbuf || !idx || !out)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_varlen: null pointer");
+  if (!aligned16(q) || !aligned16(kbuf) || !aligned16(vbuf) || !aligned16(idx) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_varlen: pointers must be 16-byte aligned");
+  if (n_h < 1 || D_qk < 1 || D_v < 1 || k < 1)
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_varlen: sizes must be positive");
+  if (k_row_stride < D_qk || v_row_stride < D_v || (k_row_stride % 8) || (v_row_stride % 8))
+    return set_error(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_varlen: row strides must cover the row and be multiples of 8");
+  return sparse_attn_launch(q, kbuf, k_row_stride, vbuf, v_row_stride, idx, vl->B, vl->max_Lq, vl->max_Lk, 0,
+                            n_h, D_qk, D_v, k, scale, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                            &va);
+}
+
+size_t indexcache_forward_varlen_workspace(const dsa_dims* d, const dsa_varlen* vl) {
+  if (!d) return 0;
+  return std::max(dsa_indexer_topk_varlen_workspace(vl, d->H_I, d->d_I, d->k),
+                  dsa_sparse_attn_varlen_workspace(vl, d->n_h, d->D_v, d->k));
+}
+
+dsa_status indexcache_forward_varlen(const char* pattern, int n_layers, const dsa_layer_io* layers,
+                                     const dsa_dims* dims, const dsa_varlen* vl, int32_t* idx_cache, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  // [IC] §1.1: the pattern rules of indexcache_forward
+  if (!pattern || n_layers < 1) return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward_varlen: empty pattern");
+  if (pattern[0] != 'F')
+    return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward_varlen: the first layer must be 'F'");
+  for (int l = 0; l < n_layers; ++l)
+    if (pattern[l] != 'F' && pattern[l] != 'S')
+      return set_error(DSA_ERR_BAD_PATTERN, "indexcache_forward_varlen: pattern entries must be 'F' or 'S'");
+  if (!layers || !dims || !idx_cache)
+    return set_error(DSA_ERR_INVALID_ARG, "indexcache_forward_varlen: null pointer");
+  dsa_status st = check_varlen_host(vl, nullptr);
+  if (st != DSA_OK) return st;
+  const dsa_dims& d = *dims;
+  if (ws_bytes < indexcache_forward_varlen_workspace(dims, vl))
+    return set_error(DSA_ERR_WORKSPACE, "indexcache_forward_varlen: workspace too small");
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_layer_io& L = layers[l];
+    if (pattern[l] == 'F') {
+      st = check_indexer_args(L.q_idx, L.k_idx, L.w, 1, vl->max_Lq, vl->max_Lk, 0, d.H_I, d.d_I, d.k, idx_cache);
+      if (st != DSA_OK) return st;
+    }
+    if (!L.q || !L.kbuf || !L.vbuf || !L.out)
+      return set_error(DSA_ERR_INVALID_ARG, "indexcache_forward_varlen: null attention pointer");
+  }
+  // [IC] §1.2, Figure 2, per sequence of the batch
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_layer_io& L = layers[l];
+    if (pattern[l] == 'F') {
+      st = dsa_indexer_topk_varlen(L.q_idx, L.k_idx, L.w, vl, d.H_I, d.d_I, d.k, idx_cache, ws, ws_bytes, stream);
+      if (st != DSA_OK) return st;
+    }
+    st = dsa_sparse_attn_varlen(L.q, L.kbuf, d.k_row_stride, L.vbuf, d.v_row_stride, idx_cache, vl, d.n_h, d.D_qk,
+                                d.D_v, d.k, d.scale, L.out, L.lse, ws, ws_bytes, stream);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_check_varlen(const dsa_varlen* vl, int* bad_seqs, void* stream) {
+  dsa_status st = check_varlen_host(vl, nullptr);
+  if (st != DSA_OK) return st;
+  if (!bad_seqs) return set_error(DSA_ERR_INVALID_ARG, "dsa_check_varlen: null pointer");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(bad_seqs, 0, sizeof(int), s);
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("dsa_check_varlen: ") + cudaGetErrorString(e));
+  const unsigned blocks = static_cast<unsigned>(std::min(1024, (vl->B + 255) / 256));
+  check_varlen_kernel<<<blocks, 256, 0, s>>>(vl->cu_q, vl->cu_k, vl->start_pos, vl->B, vl->total_q, vl->total_k,
+                                             vl->max_Lq, vl->max_Lk, bad_seqs);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("dsa_check_varlen launch: ") + cudaGetErrorString(e));
   return DSA_OK;
 }
 

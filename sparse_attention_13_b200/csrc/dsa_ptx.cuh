@@ -227,6 +227,38 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Block-scaled MMA (kind::mxf8f6f4, one ue8m0 scale per 32 elements of K):
+// D[tmem] (+)= (A * SFA) (B * SFB)^T with A, B 8-bit element codes in shared
+// memory and the scales in TMEM (sfa / sfb: column addresses; the byte within
+// the 32-bit column comes from the scale-factor ids of idesc).
+__device__ __forceinline__ void umma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Scale-factor byte ids of a block-scaled instruction descriptor (A: bits
+// 29-30, B: bits 4-5).
+__host__ __device__ constexpr uint32_t mx_sf_ids(int a_id, int b_id) {
+  return (static_cast<uint32_t>(a_id) << 29) | (static_cast<uint32_t>(b_id) << 4);
+}
+// Instruction descriptor of kind::mxf8f6f4 with ue8m0 scales, K-major A and
+// B, M rows (N is or-ed in by the caller: (N >> 3) << 17).  Element formats:
+// 0 = E4M3, 5 = E2M1 (one element per byte).
+__host__ __device__ constexpr uint32_t make_idesc_mx(int M, int fmt_a, int fmt_b) {
+  return (static_cast<uint32_t>(fmt_a) << 7) | (static_cast<uint32_t>(fmt_b) << 10) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+// Copies 32 rows x 16 bytes from shared memory into TMEM lanes 0-31 of four
+// 32-bit columns, repeated in every lane quarter (the layout block-scaled
+// MMAs read scales from: lane l, column c, byte b = row l's byte 4c + b).
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive (once) on an mbarrier when all previously issued MMAs of this
 // thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {

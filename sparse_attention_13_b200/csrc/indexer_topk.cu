@@ -43,7 +43,6 @@ constexpr int kQB = 8;        // queries per work item
 constexpr int kTileK = 128;   // keys per tile = UMMA M
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kQPT = 16 / kEpiWarps;  // queries per epilogue thread in a 4-query half
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
@@ -56,24 +55,43 @@ constexpr int kSmemBudget = 227 * 1024;
 
 __host__ __device__ constexpr int cap_for(int k) { return 3 * k + kTileK; }
 
-template <int H, int D>
+// Kernel shape.  bf16 operands: an MMA unit is one key tile against 4 queries
+// (N = 4H, two units per tile).  MX operands (the low-precision selector of
+// "注意力机制中的 Index" §5.4): 8-bit element codes, one K chunk of 128 bytes,
+// units of 2 queries (N = 2H) so that the block scales fit in TMEM beside two
+// accumulators.
+template <int H, int D, bool MX = false>
 struct Cfg {
-  static constexpr int kChunkElems = D < 64 ? D : 64;
-  static constexpr int kChunkBytes = kChunkElems * 2;
+  static constexpr int kElemBytes = MX ? 1 : 2;
+  static constexpr int kChunkElems = MX ? D : (D < 64 ? D : 64);
+  static constexpr int kChunkBytes = kChunkElems * kElemBytes;
   static constexpr int kChunks = D / kChunkElems;
   static constexpr uint32_t kSwz = kChunkBytes == 128 ? kSwizzle128B : kSwizzle64B;
   static constexpr int kSBO = 8 * kChunkBytes;
-  static constexpr int kHalfRows = 4 * H;                        // q rows of 4 queries
-  static constexpr int kQHalfBytes = kHalfRows * kChunkBytes;    // one (chunk, half) block
-  static constexpr int kQBytes = kQB * H * D * 2;
+  static constexpr int kUnitQ = MX ? 2 : 4;                      // queries per MMA unit
+  static constexpr int kUnits = kQB / kUnitQ;                    // units per key tile
+  static constexpr int kQPT = kUnitQ / 2;                        // queries per epilogue thread in a unit
+  static constexpr int kUnitRows = kUnitQ * H;                   // q rows of one unit (= N)
+  static constexpr int kAccCols = kUnitRows;                     // TMEM columns of one accumulator
+  static constexpr int kQUnitBytes = kUnitRows * kChunkBytes;    // one (chunk, unit) block
+  static constexpr int kQBytes = kQB * H * D * kElemBytes;
   static constexpr int kKeyChunkBytes = kTileK * kChunkBytes;
-  static constexpr int kStageBytes = kTileK * D * 2;
-  static constexpr int kFixed = kQBytes + kQB * H * 4 + 8192;    // q + w + small state
-  static constexpr int kStagesFit = (kSmemBudget - 1024 - kFixed) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
+  static constexpr int kStageBytes = kTileK * D * kElemBytes;
+  static constexpr int kSfBytes = MX ? 512 : 0;                  // block scales of 128 rows
+  static constexpr int kFixed = kQBytes + kUnits * kSfBytes + kQB * H * 4 + 8192;  // q + w + small state
+  static constexpr int kStagesFit = (kSmemBudget - 1024 - kFixed) / (kStageBytes + kSfBytes);
+  static constexpr int kMaxStages = MX ? 6 : 4;
+  static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
+  // MX TMEM: accumulators [0, 2 kAccCols), key scales SFA[2] (4 columns each,
+  // by tile parity), query scales SFB[2][kUnits] (4 columns each, by item parity)
+  static constexpr uint32_t kSfaCol = 2 * kAccCols;
+  static constexpr uint32_t kSfbCol = kSfaCol + 8;
   static_assert(kStages >= 2, "shared memory too small for two key stages");
-  static_assert(kHalfRows <= 256, "TMA box rows");
-  static_assert(kQHalfBytes % 512 == 0, "swizzle atom alignment");
+  static_assert(kUnitRows <= 256, "TMA box rows");
+  static_assert(kQUnitBytes % 512 == 0, "swizzle atom alignment");
+  static_assert(!MX || (D == 128 && H == 64), "MX operands: d_I = 128, H_I = 64");
+  static_assert(!MX || kSfbCol + 2 * kUnits * 4 <= kTmemCols, "MX TMEM layout");
+  static_assert(MX || 2 * kAccCols <= kTmemCols, "TMEM accumulators");
 };
 
 struct SelShared {
@@ -86,28 +104,51 @@ struct SelShared {
 
 struct EpiShared {
   unsigned long long thr[kQB];
+  int lim[kQB];         // per query slot: keys s < lim are candidates (0: no query row)
   int cnt[2][kQB];
   int qcount[2][kQB][4];
   SelShared sel;
 };
 
 struct Params {
-  const float* w;        // [B, Lq, H]
-  int32_t* idx;          // [B, Lq, k]
+  const float* w;        // [rows, H]
+  int32_t* idx;          // [rows, k]
   uint64_t* cand;        // [grid][kQB][cap]
-  uint64_t* split_out;   // [B*Lq][S][k]
-  int* split_cnt;        // [B*Lq][S]
+  uint64_t* split_out;   // [rows][S][k]
+  int* split_cnt;        // [rows][S]
   unsigned int* err;     // device error word
-  int B, Lq, Lk, start_pos, k, cap;
+  // Variable-length batches (all three null for a uniform batch): sequence
+  // b's query rows are cu_q[b] .. cu_q[b+1]-1 of the packed tensors, its keys
+  // rows cu_k[b] .. cu_k[b+1]-1, and its first query row sits at sp[b].
+  const int* cu_q;
+  const int* cu_k;
+  const int* sp;
+  int B, Lq, Lk, start_pos, k, cap;  // Lq, Lk: the maxima over the batch when varlen
   int S, split_len, n_qblocks, n_items;
+  // MX operands (uniform batches): block scales in the TMEM-copy layout, 512
+  // bytes per group of 128 rows (query rows of one batch: [sfq_groups], key
+  // rows: [sfk_tiles]); the block-scaled instruction descriptor without N.
+  const uint8_t* sfq;
+  const uint8_t* sfk;
+  int sfq_groups, sfk_tiles;
+  uint32_t mx_idesc;
 };
 
 struct Item {
   int b, qb, split;
   int s_begin, s_end;   // key range [s_begin, s_end) scanned by this item
   int n_tiles;
-  int nq[2];            // valid queries per half
+  int nvalid;           // valid queries of the block (may be <= 0 past the sequence)
+  int lq, start;        // the sequence's query rows and its first row's position
+  int q_row0, k_row0;   // first query / key row of the sequence in the q / k tensor maps
+  int tb;               // batch coordinate of the tensor maps
+  size_t out_row0;      // row of the sequence's first query in w, idx and the split lists
 };
+
+// valid queries of MMA unit u (unitq queries per unit)
+__device__ __forceinline__ int unit_queries(const Item& it, int u, int unitq) {
+  return max(0, min(unitq, it.nvalid - unitq * u));
+}
 
 __device__ __forceinline__ Item decode_item(const Params& p, int w) {
   Item it;
@@ -115,14 +156,29 @@ __device__ __forceinline__ Item decode_item(const Params& p, int w) {
   const int rest = w / p.S;
   it.b = rest % p.B;
   it.qb = p.n_qblocks - 1 - rest / p.B;  // longest query blocks first
+  if (p.cu_q) {
+    const int q0 = __ldg(p.cu_q + it.b);
+    it.lq = min(max(__ldg(p.cu_q + it.b + 1) - q0, 0), p.Lq);
+    it.start = max(__ldg(p.sp + it.b), 0);
+    it.q_row0 = q0;
+    it.k_row0 = __ldg(p.cu_k + it.b);
+    it.tb = 0;
+    it.out_row0 = static_cast<size_t>(q0);
+  } else {
+    it.lq = p.Lq;
+    it.start = p.start_pos;
+    it.q_row0 = 0;
+    it.k_row0 = 0;
+    it.tb = it.b;
+    it.out_row0 = static_cast<size_t>(it.b) * p.Lq;
+  }
   const int i0 = it.qb * kQB;
-  const int nvalid = min(kQB, p.Lq - i0);
-  it.nq[0] = max(0, min(4, nvalid));
-  it.nq[1] = max(0, min(4, nvalid - 4));
-  const int t_max = p.start_pos + i0 + nvalid - 1;  // largest visible count in the block
+  const int nvalid = min(kQB, it.lq - i0);
+  it.nvalid = nvalid;
+  const int t_max = it.start + i0 + nvalid - 1;  // largest visible count in the block
   it.s_begin = it.split * p.split_len;
   it.s_end = min(t_max, it.s_begin + p.split_len);
-  it.n_tiles = it.s_end > it.s_begin ? (it.s_end - it.s_begin + kTileK - 1) / kTileK : 0;
+  it.n_tiles = nvalid > 0 && it.s_end > it.s_begin ? (it.s_end - it.s_begin + kTileK - 1) / kTileK : 0;
   return it;
 }
 
@@ -306,17 +362,20 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
 }
 
 // ------------------------------------------------------------------ kernel
-template <int H, int D>
+template <int H, int D, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const Params p) {
-  using C = Cfg<H, D>;
+  using C = Cfg<H, D, MX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* q_smem = smem;
   uint8_t* key_smem = q_smem + C::kQBytes;
-  float* w_smem = reinterpret_cast<float*>(key_smem + C::kStages * C::kStageBytes);
+  // MX: the query block's scales (kUnits x 512 B), then one 512 B block per key stage
+  uint8_t* sfq_smem = key_smem + C::kStages * C::kStageBytes;
+  uint8_t* sfk_smem = sfq_smem + C::kUnits * C::kSfBytes;
+  float* w_smem = reinterpret_cast<float*>(sfk_smem + C::kStages * C::kSfBytes);
   EpiShared* es = reinterpret_cast<EpiShared*>(w_smem + kQB * H);
   uint64_t* bars = reinterpret_cast<uint64_t*>(es + 1);
   uint64_t* key_full = bars;
@@ -372,19 +431,26 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
         const Item it = decode_item(p, w);
         if (it.n_tiles == 0) continue;
         if (!mbar_wait(q_empty, (n_items_done & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(q_full, C::kQBytes);
+        mbar_arrive_expect_tx(q_full, C::kQBytes + C::kUnits * C::kSfBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          for (int h = 0; h < 2; ++h)
-            tma_load_3d(q_smem + (c * 2 + h) * C::kQHalfBytes, &tm_q, q_full,
-                        c * C::kChunkElems, (it.qb * kQB + 4 * h) * H, it.b);
+          for (int h = 0; h < C::kUnits; ++h)
+            tma_load_3d(q_smem + (c * C::kUnits + h) * C::kQUnitBytes, &tm_q, q_full,
+                        c * C::kChunkElems, (it.q_row0 + it.qb * kQB + C::kUnitQ * h) * H, it.tb);
+        if constexpr (MX)  // the block's kUnits scale groups are contiguous
+          bulk_load_g2s(sfq_smem, p.sfq + (static_cast<size_t>(it.tb) * p.sfq_groups + it.qb * C::kUnits) * 512,
+                        C::kUnits * C::kSfBytes, q_full);
         bool ok = true;
         for (int j = 0; j < it.n_tiles; ++j) {
           if (!mbar_wait(&key_empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&key_full[stage], C::kStageBytes);
+          mbar_arrive_expect_tx(&key_full[stage], C::kStageBytes + C::kSfBytes);
           uint8_t* dst = key_smem + stage * C::kStageBytes;
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_3d(dst + c * C::kKeyChunkBytes, &tm_k, &key_full[stage],
-                        c * C::kChunkElems, it.s_begin + j * kTileK, it.b);
+                        c * C::kChunkElems, it.k_row0 + it.s_begin + j * kTileK, it.tb);
+          if constexpr (MX)
+            bulk_load_g2s(sfk_smem + stage * C::kSfBytes,
+                          p.sfk + (static_cast<size_t>(it.tb) * p.sfk_tiles + (it.s_begin + j * kTileK) / kTileK) * 512,
+                          C::kSfBytes, &key_full[stage]);
           ++issued_tiles;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
@@ -408,28 +474,52 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (it.n_tiles == 0) continue;
         if (!mbar_wait(q_full, n_items_done & 1, abort_flag)) break;
         tc_fence_after();
+        const uint32_t sfb_col = C::kSfbCol + (n_items_done & 1) * C::kUnits * 4;
+        if constexpr (MX) {
+          // the query block's scales into TMEM (this item's parity): tcgen05
+          // copies and MMAs of one thread run in issue order
+          for (int h = 0; h < C::kUnits; ++h)
+            tc_cp_32x128b_x4(tmem_base + sfb_col + 4 * h,
+                             make_smem_desc(smem_u32(sfq_smem + h * C::kSfBytes), 16, 128, kSwizzleNone));
+        }
         for (int j = 0; j < it.n_tiles && ok; ++j) {
           if (!mbar_wait(&key_full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(key_smem + stage * C::kStageBytes);
-          for (int h = 0; h < 2; ++h) {
-            if (it.nq[h] == 0) continue;
+          const uint32_t sfa_col = C::kSfaCol + (*consumed_tiles & 1) * 4;
+          if constexpr (MX)
+            tc_cp_32x128b_x4(tmem_base + sfa_col,
+                             make_smem_desc(smem_u32(sfk_smem + stage * C::kSfBytes), 16, 128, kSwizzleNone));
+          for (int h = 0; h < C::kUnits; ++h) {
+            if (unit_queries(it, h, C::kUnitQ) == 0) continue;
             const uint32_t buf = unit & 1;
             if (!mbar_wait(&tmem_empty[buf], ((unit >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const int n = ((it.nq[h] * H + 15) / 16) * 16;
-            const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
-            const uint32_t d_tmem = tmem_base + buf * 256;
-            const uint32_t b_base = smem_u32(q_smem) + h * C::kQHalfBytes;
+            const int n = ((unit_queries(it, h, C::kUnitQ) * H + 15) / 16) * 16;
+            const uint32_t d_tmem = tmem_base + buf * C::kAccCols;
+            const uint32_t b_base = smem_u32(q_smem) + h * C::kQUnitBytes;
+            if constexpr (MX) {
+              // four K = 32 steps; step kk takes byte kk of the scale columns
+              const uint32_t idesc = p.mx_idesc | (static_cast<uint32_t>(n >> 3) << 17);
 #pragma unroll
-            for (int c = 0; c < C::kChunks; ++c) {
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = make_smem_desc(a_base + kk * 32, 16, C::kSBO, C::kSwz);
+                const uint64_t bd = make_smem_desc(b_base + kk * 32, 16, C::kSBO, C::kSwz);
+                umma_mx_ss(d_tmem, ad, bd, idesc | mx_sf_ids(kk, kk), tmem_base + sfa_col,
+                           tmem_base + sfb_col + 4 * h, kk != 0);
+              }
+            } else {
+              const uint32_t idesc = make_idesc_bf16(128, n, 0, 0);
 #pragma unroll
-              for (int kk = 0; kk < C::kChunkElems / 16; ++kk) {
-                const uint64_t ad = make_smem_desc(a_base + c * C::kKeyChunkBytes + kk * 32, 16,
-                                                   C::kSBO, C::kSwz);
-                const uint64_t bd = make_smem_desc(b_base + c * 2 * C::kQHalfBytes + kk * 32, 16,
-                                                   C::kSBO, C::kSwz);
-                umma_bf16_ss(d_tmem, ad, bd, idesc, (c | kk) != 0);
+              for (int c = 0; c < C::kChunks; ++c) {
+#pragma unroll
+                for (int kk = 0; kk < C::kChunkElems / 16; ++kk) {
+                  const uint64_t ad = make_smem_desc(a_base + c * C::kKeyChunkBytes + kk * 32, 16,
+                                                     C::kSBO, C::kSwz);
+                  const uint64_t bd = make_smem_desc(b_base + c * C::kUnits * C::kQUnitBytes + kk * 32, 16,
+                                                     C::kSBO, C::kSwz);
+                  umma_bf16_ss(d_tmem, ad, bd, idesc, (c | kk) != 0);
+                }
               }
             }
             umma_commit(&tmem_full[buf]);
@@ -459,11 +549,13 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (tid < kQB) {
         es->thr[tid] = 0ull;
         es->cnt[0][tid] = 0;
+        // row i0 + tid sees s < t = start + i0 + tid, within this item's key range
+        es->lim[tid] = i0 + tid < it.lq ? min(it.start + i0 + tid, it.s_end) : 0;
       }
       for (int e = tid; e < kQB * H; e += kEpiThreads) {
         const int qs = e / H;
         const int i = i0 + qs;
-        w_smem[e] = i < p.Lq ? p.w[(static_cast<size_t>(it.b) * p.Lq + i) * H + (e % H)] : 0.f;
+        w_smem[e] = i < it.lq ? p.w[(it.out_row0 + i) * H + (e % H)] : 0.f;
       }
       named_bar_sync(kEpiBar, kEpiThreads);
       uint64_t* cand_base = p.cand + static_cast<size_t>(cta) * kQB * p.cap;
@@ -471,20 +563,20 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int j = 0; j < it.n_tiles && ok; ++j) {
         const int par = j & 1;
         const int s = it.s_begin + j * kTileK + qd * 32 + lane;
-        for (int h = 0; h < 2; ++h) {
-          if (it.nq[h] == 0) continue;
+        for (int h = 0; h < C::kUnits; ++h) {
+          if (unit_queries(it, h, C::kUnitQ) == 0) continue;
           const uint32_t buf = unit & 1;
           if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[buf], (unit >> 1) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
-          float acc[kQPT];
-          const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + buf * 256;
+          float acc[C::kQPT];
+          const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + buf * C::kAccCols;
           if constexpr (H >= 32) {
-            uint32_t v[kQPT][H];
+            uint32_t v[C::kQPT][H];
 #pragma unroll
-            for (int jj = 0; jj < kQPT; ++jj)
+            for (int jj = 0; jj < C::kQPT; ++jj)
 #pragma unroll
               for (int c = 0; c < H / 32; ++c)
-                tmem_ld32<32>(t_lane + (kQPT * qg + jj) * H + c * 32,
+                tmem_ld32<32>(t_lane + (C::kQPT * qg + jj) * H + c * 32,
                               *reinterpret_cast<uint32_t(*)[32]>(&v[jj][c * 32]));
             tmem_ld_wait();
             tc_fence_before();
@@ -493,8 +585,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
             // heads j = 4c + r accumulate into a[r] (four independent FMA
             // chains), combined as (a0 + a1) + (a2 + a3)
 #pragma unroll
-            for (int jj = 0; jj < kQPT; ++jj) {
-              const float4* w4 = reinterpret_cast<const float4*>(w_smem + (4 * h + kQPT * qg + jj) * H);
+            for (int jj = 0; jj < C::kQPT; ++jj) {
+              const float4* w4 = reinterpret_cast<const float4*>(w_smem + (C::kUnitQ * h + C::kQPT * qg + jj) * H);
               float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < H / 4; ++c) {
@@ -507,32 +599,36 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
               acc[jj] = (a[0] + a[1]) + (a[2] + a[3]);
             }
           } else {
-            uint32_t v[kQPT][H];
+            uint32_t v[C::kQPT][H];
 #pragma unroll
-            for (int jj = 0; jj < kQPT; ++jj)
-              tmem_ld32<H>(t_lane + (kQPT * qg + jj) * H, v[jj]);
+            for (int jj = 0; jj < C::kQPT; ++jj)
+              tmem_ld32<H>(t_lane + (C::kQPT * qg + jj) * H, v[jj]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_empty[buf]);
 #pragma unroll
-            for (int jj = 0; jj < kQPT; ++jj) {
-              const float* wq = w_smem + (4 * h + kQPT * qg + jj) * H;
+            for (int jj = 0; jj < C::kQPT; ++jj) {
+              const float* wq = w_smem + (C::kUnitQ * h + C::kQPT * qg + jj) * H;
               float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < H; ++c) a[c & 3] = fmaf(fmaxf(__uint_as_float(v[jj][c]), 0.f), wq[c], a[c & 3]);
               acc[jj] = (a[0] + a[1]) + (a[2] + a[3]);
             }
           }
-          // candidate test and ordered append
-          unsigned long long P[kQPT];
-          unsigned msk[kQPT];
+          if constexpr (MX) {
+            // the low-precision selector ranks scores quantised from fp32 to
+            // bf16 (round to nearest even)
 #pragma unroll
-          for (int jj = 0; jj < kQPT; ++jj) {
-            const int qs = 4 * h + kQPT * qg + jj;
-            const int i = i0 + qs;
-            const int T = p.start_pos + i;
-            const bool valid = (i < p.Lq) && (s < T) && (s < it.s_end);
+            for (int jj = 0; jj < C::kQPT; ++jj) acc[jj] = __bfloat162float(__float2bfloat16_rn(acc[jj]));
+          }
+          // candidate test and ordered append
+          unsigned long long P[C::kQPT];
+          unsigned msk[C::kQPT];
+#pragma unroll
+          for (int jj = 0; jj < C::kQPT; ++jj) {
+            const int qs = C::kUnitQ * h + C::kQPT * qg + jj;
+            const bool valid = s < es->lim[qs];
             P[jj] = pack_entry(acc[jj], s);
             const bool cand = valid && P[jj] > es->thr[qs];
             msk[jj] = __ballot_sync(0xffffffffu, cand);
@@ -541,8 +637,8 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
           named_bar_sync(kEpiBar, kEpiThreads);
           bool need_sel = false;
 #pragma unroll
-          for (int jj = 0; jj < kQPT; ++jj) {
-            const int qs = 4 * h + kQPT * qg + jj;
+          for (int jj = 0; jj < C::kQPT; ++jj) {
+            const int qs = C::kUnitQ * h + C::kQPT * qg + jj;
             const int base = es->cnt[par][qs];
             int off = base;
             for (int x = 0; x < qd; ++x) off += es->qcount[par][qs][x];
@@ -550,22 +646,22 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
               cand_base[static_cast<size_t>(qs) * p.cap + off + __popc(msk[jj] & ((1u << lane) - 1u))] = P[jj];
             }
           }
-          // every thread derives the new counts of the half's 4 queries
-          int newcnt[4];
+          // every thread derives the new counts of the unit's queries
+          int newcnt[C::kUnitQ];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int qs = 4 * h + q4;
+          for (int q4 = 0; q4 < C::kUnitQ; ++q4) {
+            const int qs = C::kUnitQ * h + q4;
             newcnt[q4] = es->cnt[par][qs] + es->qcount[par][qs][0] + es->qcount[par][qs][1] +
                          es->qcount[par][qs][2] + es->qcount[par][qs][3];
             need_sel |= newcnt[q4] > p.cap - kTileK;
           }
-          if (tid < 4) es->cnt[par ^ 1][4 * h + tid] = newcnt[tid];
+          if (tid < C::kUnitQ) es->cnt[par ^ 1][C::kUnitQ * h + tid] = newcnt[tid];
           if (need_sel) {
             named_bar_sync(kEpiBar, kEpiThreads);  // appends and counts visible
 #pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < C::kUnitQ; ++q4) {
               if (newcnt[q4] <= p.cap - kTileK) continue;
-              const int qs = 4 * h + q4;
+              const int qs = C::kUnitQ * h + q4;
               uint64_t* bq = cand_base + static_cast<size_t>(qs) * p.cap;
               const unsigned long long kth =
                   select_topk(bq, bq, newcnt[q4], p.k, 0, nullptr, nullptr, nullptr, es->sel);
@@ -580,20 +676,22 @@ indexer_topk_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       if (!ok) break;
-      // final selection per query row
+      // final selection per query row (the item's placement is decoded again
+      // here rather than kept in registers through the tile loop)
       named_bar_sync(kEpiBar, kEpiThreads);
       const int fpar = it.n_tiles & 1;
+      const Item itf = decode_item(p, w);
 #pragma unroll 1
       for (int qs = 0; qs < kQB; ++qs) {
         const int i = i0 + qs;
-        if (i >= p.Lq) break;
+        if (i >= itf.lq) break;
         const int c = es->cnt[fpar][qs];
         const uint64_t* bq = cand_base + static_cast<size_t>(qs) * p.cap;
-        const size_t row = static_cast<size_t>(it.b) * p.Lq + i;
+        const size_t row = itf.out_row0 + i;
         if (p.S == 1) {
           select_topk(bq, nullptr, c, p.k, 1, p.idx + row * p.k, nullptr, nullptr, es->sel);
         } else {
-          const size_t slot = row * p.S + it.split;
+          const size_t slot = row * p.S + itf.split;
           select_topk(bq, nullptr, c, p.k, 2, nullptr, p.split_out + slot * p.k,
                       p.split_cnt + slot, es->sel);
         }
@@ -785,15 +883,16 @@ indexer_merge_kernel(const uint64_t* __restrict__ split_out, const int* __restri
   for (int q = total + tid; q < k; q += kMergeThreads) out[q] = -1;
 }
 
-template <int H, int D>
+template <int H, int D, bool MX = false>
 dsa_status launch_hd(const CUtensorMap& tq, const CUtensorMap& tk, const Params& p, int grid,
                      cudaStream_t stream) {
-  using C = Cfg<H, D>;
+  using C = Cfg<H, D, MX>;
   // At least 120 KB so that one CTA owns each SM (and all of its TMEM).
   const int smem = std::max(120 * 1024, 1024 + C::kQBytes + C::kStages * C::kStageBytes +
+                                            (C::kUnits + C::kStages) * C::kSfBytes +
                                             kQB * H * 4 + static_cast<int>(sizeof(EpiShared)) +
                                             (2 * C::kStages + 6) * 8 + 32);
-  auto kern = indexer_topk_kernel<H, D>;
+  auto kern = indexer_topk_kernel<H, D, MX>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("indexer smem attribute: ") + cudaGetErrorString(e));
   e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tq, tk, p);
@@ -810,7 +909,7 @@ bool indexer_supported(int H, int d, int k) {
   return h_ok && d_ok && k >= 1 && k <= kMaxK;
 }
 
-IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k) {
+IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k, long long rows_in) {
   (void)Lk;
   IndexerPlan pl{};
   pl.n_qblocks = (Lq + kQB - 1) / kQB;
@@ -830,19 +929,42 @@ IndexerPlan indexer_plan(int B, int Lq, int Lk, int start_pos, int k) {
   pl.grid = std::min(pl.n_items, kMaxGrid);
   pl.cap = cap_for(k);
   pl.cand_bytes = static_cast<size_t>(kMaxGrid) * kQB * pl.cap * 8;
-  const size_t rows = static_cast<size_t>(B) * Lq;
+  const size_t rows = rows_in >= 0 ? static_cast<size_t>(rows_in) : static_cast<size_t>(B) * Lq;
   pl.split_bytes = S > 1 ? rows * S * k * 8 : 0;
   pl.split_cnt_bytes = S > 1 ? ((rows * S * 4 + 255) / 256) * 256 : 0;
   pl.total_bytes = pl.cand_bytes + pl.split_bytes + pl.split_cnt_bytes;
   return pl;
 }
 
+// Decode rows of a varlen batch: one query row per sequence (max_Lq = 1 and
+// total_q = B) against caches the decode kernels can slice.
+static bool varlen_decode_applies(int B, int max_Lq, int max_Lk, int total_q, int H, int d) {
+  return max_Lq == 1 && total_q == B && decode_indexer_applies(1, max_Lk, max_Lk, H, d);
+}
+
+size_t indexer_varlen_ws_bytes(int B, int max_Lq, int max_Lk, int total_q, int H, int d, int k) {
+  if (varlen_decode_applies(B, max_Lq, max_Lk, total_q, H, d)) return decode_indexer_ws_bytes(B, max_Lk);
+  // every row sees at most max_Lk positions
+  return indexer_plan(B, max_Lq, max_Lk, std::max(0, max_Lk - max_Lq + 1), std::min(k, kMaxK), total_q)
+      .total_bytes;
+}
+
 dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, const float* w,
                                int B, int Lq, int Lk, int start_pos, int H, int d, int k,
-                               int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (decode_indexer_applies(Lq, Lk, start_pos, H, d) && ws_bytes >= decode_indexer_ws_bytes(B, Lk))
+                               int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream,
+                               const VarlenArgs* vl) {
+  if (vl) {
+    if (varlen_decode_applies(B, Lq, Lk, vl->total_q, H, d) && ws_bytes >= decode_indexer_ws_bytes(B, Lk)) {
+      const DecodeVarlen dv{vl->sp, vl->cu_k, vl->total_k};
+      return decode_indexer_launch(q_idx, k_idx, w, B, Lk, 0, H, d, k, idx, ws, ws_bytes, stream, &dv);
+    }
+    // the plan covers rows up to t = Lk (no row sees more than its cache)
+    start_pos = std::max(0, Lk - Lq + 1);
+  } else if (decode_indexer_applies(Lq, Lk, start_pos, H, d) && ws_bytes >= decode_indexer_ws_bytes(B, Lk)) {
     return decode_indexer_launch(q_idx, k_idx, w, B, Lk, start_pos, H, d, k, idx, ws, ws_bytes, stream);
-  IndexerPlan pl = indexer_plan(B, Lq, Lk, start_pos, k);
+  }
+  const long long rows = vl ? static_cast<long long>(vl->total_q) : static_cast<long long>(B) * Lq;
+  IndexerPlan pl = indexer_plan(B, Lq, Lk, start_pos, k, rows);
   if (ws_bytes < pl.total_bytes) return set_error(DSA_ERR_WORKSPACE, "indexer workspace too small");
   const int sms = device_sm_count();
   if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
@@ -851,11 +973,13 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
   const int chunk = d < 64 ? d : 64;
   const CUtensorMapSwizzle swz = chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap tq, tk;
-  if (!encode_tiled_3d(&tq, q_idx, d, static_cast<uint64_t>(Lq) * H, B, static_cast<uint64_t>(d) * 2,
-                       static_cast<uint64_t>(Lq) * H * d * 2, chunk, 4 * H, swz))
+  // uniform: [B][Lq * H][d] and [B][Lk][d]; varlen: one batch of the packed rows
+  const uint64_t qrows = vl ? static_cast<uint64_t>(vl->total_q) * H : static_cast<uint64_t>(Lq) * H;
+  const uint64_t krows = vl ? static_cast<uint64_t>(vl->total_k) : static_cast<uint64_t>(Lk);
+  const uint64_t nb = vl ? 1u : static_cast<uint64_t>(B);
+  if (!encode_tiled_3d(&tq, q_idx, d, qrows, nb, static_cast<uint64_t>(d) * 2, qrows * d * 2, chunk, 4 * H, swz))
     return set_error(DSA_ERR_CUDA, "tensor map for q_idx failed");
-  if (!encode_tiled_3d(&tk, k_idx, d, Lk, B, static_cast<uint64_t>(d) * 2,
-                       static_cast<uint64_t>(Lk) * d * 2, chunk, kTileK, swz))
+  if (!encode_tiled_3d(&tk, k_idx, d, krows, nb, static_cast<uint64_t>(d) * 2, krows * d * 2, chunk, kTileK, swz))
     return set_error(DSA_ERR_CUDA, "tensor map for k_idx failed");
 
   Params p{};
@@ -867,12 +991,15 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
   p.split_cnt = pl.S > 1 ? reinterpret_cast<int*>(base + pl.cand_bytes + pl.split_bytes) : nullptr;
   p.err = device_error_word();
   if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+  p.cu_q = vl ? vl->cu_q : nullptr;
+  p.cu_k = vl ? vl->cu_k : nullptr;
+  p.sp = vl ? vl->sp : nullptr;
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k; p.cap = pl.cap;
   p.S = pl.S; p.split_len = pl.split_len; p.n_qblocks = pl.n_qblocks; p.n_items = pl.n_items;
 
   dsa_status st = DSA_ERR_UNSUPPORTED;
 #define DSA_CASE(HH, DD) \
-  if (H == HH && d == DD) st = launch_hd<HH, DD>(tq, tk, p, grid, stream);
+  if (H == HH && d == DD) st = launch_hd<HH, DD, false>(tq, tk, p, grid, stream);
   DSA_CASE(4, 32) DSA_CASE(4, 64) DSA_CASE(4, 128)
   DSA_CASE(8, 32) DSA_CASE(8, 64) DSA_CASE(8, 128)
   DSA_CASE(16, 32) DSA_CASE(16, 64) DSA_CASE(16, 128)
@@ -886,8 +1013,63 @@ dsa_status indexer_topk_launch(const dsa_bf16* q_idx, const dsa_bf16* k_idx, con
       cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(indexer_merge_kernel), msmem);
       if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge smem attribute: ") + cudaGetErrorString(e));
     }
-    cudaError_t e = launch_pdl(indexer_merge_kernel, dim3(static_cast<unsigned>(static_cast<size_t>(B) * Lq)),
+    cudaError_t e = launch_pdl(indexer_merge_kernel, dim3(static_cast<unsigned>(rows)),
                                dim3(kMergeThreads), msmem, stream, p.split_out, p.split_cnt, idx, pl.S, k);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge launch: ") + cudaGetErrorString(e));
+  }
+  return DSA_OK;
+}
+
+// The low-precision selector ("注意力机制中的 Index" §5.4): the same fused
+// indexer + top-k over MX operands (H_I = 64, d_I = 128, uniform batches).
+// codes_q [B][Lq * 64][128] and codes_k [B][Lk][128] hold one element code
+// per byte; sfq [B][sfq_groups] and sfk [B][sfk_tiles] hold the block scales
+// of each group of 128 rows in the layout the TMEM copy reads (row 32c + l of
+// the group, block n at byte 16 l + 4 c + n).  The workspace starts with the
+// plan's candidate and split buffers.
+dsa_status indexer_topk_mx_launch(const uint8_t* codes_q, const uint8_t* codes_k, const uint8_t* sfq,
+                                  const uint8_t* sfk, int sfq_groups, int sfk_tiles, const float* w, int B, int Lq,
+                                  int Lk, int start_pos, int fmt_code, int k, int32_t* idx, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream) {
+  constexpr int H = 64, d = 128;
+  const long long rows = static_cast<long long>(B) * Lq;
+  IndexerPlan pl = indexer_plan(B, Lq, Lk, start_pos, k, rows);
+  if (ws_bytes < pl.total_bytes) return set_error(DSA_ERR_WORKSPACE, "low-precision indexer workspace too small");
+  const int sms = device_sm_count();
+  if (sms <= 0) return set_error(DSA_ERR_CUDA, "cannot query the device SM count");
+  const int grid = std::max(1, std::min(pl.grid, sms));
+  CUtensorMap tq, tk;
+  const uint64_t qrows = static_cast<uint64_t>(Lq) * H;
+  if (!encode_tiled_3d(&tq, codes_q, d, qrows, B, d, qrows * d, d, Cfg<H, d, true>::kUnitRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return set_error(DSA_ERR_CUDA, "tensor map for the query codes failed");
+  if (!encode_tiled_3d(&tk, codes_k, d, Lk, B, d, static_cast<uint64_t>(Lk) * d, d, kTileK,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return set_error(DSA_ERR_CUDA, "tensor map for the key codes failed");
+  Params p{};
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p.w = w;
+  p.idx = idx;
+  p.cand = reinterpret_cast<uint64_t*>(base);
+  p.split_out = pl.S > 1 ? reinterpret_cast<uint64_t*>(base + pl.cand_bytes) : nullptr;
+  p.split_cnt = pl.S > 1 ? reinterpret_cast<int*>(base + pl.cand_bytes + pl.split_bytes) : nullptr;
+  p.err = device_error_word();
+  if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k; p.cap = pl.cap;
+  p.S = pl.S; p.split_len = pl.split_len; p.n_qblocks = pl.n_qblocks; p.n_items = pl.n_items;
+  p.sfq = sfq; p.sfk = sfk; p.sfq_groups = sfq_groups; p.sfk_tiles = sfk_tiles;
+  p.mx_idesc = make_idesc_mx(128, fmt_code, fmt_code);
+  dsa_status st = launch_hd<H, d, true>(tq, tk, p, grid, stream);
+  if (st != DSA_OK) return st;
+  if (pl.S > 1) {
+    const int msmem = pl.S * k * 4;
+    if (msmem > 48 * 1024) {
+      cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(indexer_merge_kernel), msmem);
+      if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge smem attribute: ") + cudaGetErrorString(e));
+    }
+    cudaError_t e = launch_pdl(indexer_merge_kernel, dim3(static_cast<unsigned>(rows)), dim3(kMergeThreads), msmem,
+                               stream, p.split_out, p.split_cnt, idx, pl.S, k);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("merge launch: ") + cudaGetErrorString(e));
   }

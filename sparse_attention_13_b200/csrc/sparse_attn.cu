@@ -53,6 +53,44 @@ namespace dsa {
 
 namespace {
 
+// Sequence of a packed query row in a variable-length batch: the last b in
+// [0, B) with cu_q[b] <= row (empty sequences share their successor's
+// start, and the last of them owns the rows).
+__device__ __forceinline__ int seq_of_row(const int* __restrict__ cu_q, int B, int row) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu_q + mid) <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Where query row `row` sits: its sequence's first cached row, the cache
+// length and the row's absolute position t.  Uniform batch (cu_q null): row
+// = b * Lq + i at t = start_pos + i over rows b * Lk ...; varlen: from the
+// prefix arrays.
+struct RowPlace {
+  int b, t, lk;
+  long long kv_row0;
+};
+__device__ __forceinline__ RowPlace place_row(int row, int B, int Lq, int Lk, int start_pos, const int* cu_q,
+                                              const int* cu_k, const int* sp) {
+  RowPlace r;
+  if (cu_q) {
+    r.b = seq_of_row(cu_q, B, row);
+    const int k0 = __ldg(cu_k + r.b);
+    r.t = max(__ldg(sp + r.b), 0) + (row - __ldg(cu_q + r.b));
+    r.lk = __ldg(cu_k + r.b + 1) - k0;
+    r.kv_row0 = k0;
+  } else {
+    r.b = row / Lq;
+    r.t = start_pos + row % Lq;
+    r.lk = Lk;
+    r.kv_row0 = static_cast<long long>(r.b) * Lk;
+  }
+  return r;
+}
+
 // ------------------------------------------------------------------ SIMT
 constexpr int kSimtThreads = 128;
 
@@ -61,29 +99,28 @@ simt_sparse_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
                         int64_t ks, const __nv_bfloat16* __restrict__ vb, int64_t vs,
                         const int32_t* __restrict__ idx, int B, int Lq, int Lk, int start_pos,
                         int n_h, int Dqk, int Dv, int k, float scale, __nv_bfloat16* __restrict__ out,
-                        float* __restrict__ lse) {
+                        float* __restrict__ lse, const int* __restrict__ cu_q, const int* __restrict__ cu_k,
+                        const int* __restrict__ sp) {
   extern __shared__ float qs[];  // [n_h][Dqk]
   pdl_trigger();
   pdl_wait();
   const size_t row = blockIdx.x;
-  const int b = static_cast<int>(row / Lq);
-  const int i = static_cast<int>(row % Lq);
-  const int T = start_pos + i;
-  const int nv = min(T, k);
+  const RowPlace pl = place_row(static_cast<int>(row), B, Lq, Lk, start_pos, cu_q, cu_k, sp);
+  const int nv = max(0, min(pl.t, k));
   for (int e = threadIdx.x; e < n_h * Dqk; e += kSimtThreads)
     qs[e] = __bfloat162float(q[row * n_h * Dqk + e]);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* irow = idx + row * k;
-  const __nv_bfloat16* kbase = kb + static_cast<int64_t>(b) * Lk * ks;
-  const __nv_bfloat16* vbase = vb + static_cast<int64_t>(b) * Lk * vs;
+  const __nv_bfloat16* kbase = kb + pl.kv_row0 * ks;
+  const __nv_bfloat16* vbase = vb + pl.kv_row0 * vs;
   const float sl2 = scale * 1.4426950408889634f;
   for (int h = warp; h < n_h; h += kSimtThreads / 32) {
     float m = -INFINITY, l = 0.f;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < nv; ++r) {
       const int s = irow[r];
-      if (s < 0 || s >= Lk) continue;  // padding, or a position outside the sequence: skipped
+      if (s < 0 || s >= pl.lk) continue;  // padding, or a position outside the sequence: skipped
       const __nv_bfloat16* kr = kbase + static_cast<int64_t>(s) * ks;
       float dot = 0.f;
       for (int c = lane; c < Dqk; c += 32) dot += qs[h * Dqk + c] * __bfloat162float(kr[c]);
@@ -158,23 +195,30 @@ struct MlaParams {
   uint32_t* part_o;         // split partials, bf16 pairs: [B*Lq][S][256 column pairs][128 heads]
   float* part_lse;          // [B*Lq][S][128]
   unsigned int* err;
+  const int* cu_q;          // variable-length batch (null: uniform)
+  const int* cu_k;
+  const int* sp;
   int B, Lq, Lk, start_pos, k;
+  int rows;                 // query rows of the batch (B * Lq, or the packed total)
   int S, cps;               // key-range splits per row, chunks per split
   float scale_log2;
 };
 
 struct MlaItem {
-  int row, split, b, c0, n;  // chunks [c0, c0 + n) of the row's index list
+  int row, split, c0, n;     // chunks [c0, c0 + n) of the row's index list
   int nv;                    // valid index entries read: min(t, k)
+  int lk;                    // the sequence's cached rows
+  int kv_row0;               // its first latent row in the tensor map
 };
 
 __device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int item) {
   MlaItem it;
   it.row = item / p.S;
   it.split = item % p.S;
-  it.b = it.row / p.Lq;
-  const int i = it.row % p.Lq;
-  it.nv = min(p.start_pos + i, p.k);
+  const RowPlace pl = place_row(it.row, p.B, p.Lq, p.Lk, p.start_pos, p.cu_q, p.cu_k, p.sp);
+  it.nv = max(0, min(pl.t, p.k));
+  it.lk = pl.lk;
+  it.kv_row0 = static_cast<int>(pl.kv_row0);
   const int nch = (it.nv + kChunk - 1) / kChunk;
   it.c0 = it.split * p.cps;
   it.n = max(0, min(nch, it.c0 + p.cps) - it.c0);
@@ -197,7 +241,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   const uint32_t peer = rank ^ 1u;
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
-  const int n_items = p.B * p.Lq * p.S;
+  const int n_items = p.rows * p.S;
   // CTA0 owns latent columns 0..255 (QK and V), CTA1 owns 256..575 (QK) and
   // 256..511 (V); together they gather each selected row exactly once.
   const int n_slabs = rank == 0 ? 4 : 5;
@@ -252,7 +296,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       const MlaItem it = mla_item(p, item);
       if (it.n == 0) continue;
       const int32_t* irow = p.idx + static_cast<size_t>(it.row) * p.k;
-      const int row_base = it.b * p.Lk;
+      const int row_base = it.kv_row0;
       const int my_group = pw + 7 * (lane >> 2);            // group whose row this lane fetches
       auto fetch = [&](int c) -> int {
         const int r = c * kChunk + my_group * 4 + (lane & 3);
@@ -271,7 +315,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         f0 = f1;
         f1 = f2;
         f2 = c + 3 < c_end ? fetch(c + 3) : -1;
-        const bool valid = sidx >= 0 && sidx < p.Lk;
+        const bool valid = sidx >= 0 && sidx < it.lk;
         const int grow = row_base + (valid ? sidx : 0);   // padded rows read row 0 (masked later)
         const unsigned m = __ballot_sync(0xffffffffu, valid);
         const int src = (lane < n_groups ? lane : 0) * 4;
@@ -782,21 +826,25 @@ MlaSplit mla_split(long long rows, int k, int sms) {
 
 }  // namespace
 
-size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k) {
+size_t sparse_attn_ws_rows(long long rows, int n_h, int D_v, int k) {
   if (n_h != kNH || D_v != kDV) return 0;
-  const long long rows = static_cast<long long>(B) * Lq;
   // sized for up to 160 SMs so the requirement does not depend on the device
   const MlaSplit sp = mla_split(rows, k, 160);
   if (sp.S <= 1) return 0;
   return static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2 + 1) * 4 + 256;
 }
 
+size_t sparse_attn_ws_bytes(int B, int Lq, int n_h, int D_v, int k) {
+  return sparse_attn_ws_rows(static_cast<long long>(B) * Lq, n_h, D_v, k);
+}
+
 dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k_row_stride,
                               const dsa_bf16* vbuf, int64_t v_row_stride, const int32_t* idx,
                               int B, int Lq, int Lk, int start_pos, int n_h, int D_qk, int D_v,
                               int k, float scale, dsa_bf16* out, float* lse, void* ws,
-                              size_t ws_bytes, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(B) * Lq;
+                              size_t ws_bytes, cudaStream_t stream, const VarlenArgs* vl) {
+  const long long rows = vl ? static_cast<long long>(vl->total_q) : static_cast<long long>(B) * Lq;
+  const long long kv_rows = vl ? static_cast<long long>(vl->total_k) : static_cast<long long>(B) * Lk;
   if (rows > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
   const bool mla = n_h == kNH && D_qk == kDQK && D_v == kDV && kbuf == vbuf &&
                    k_row_stride == v_row_stride;
@@ -808,7 +856,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2 + 1) * 4 : 0;
     if (need > ws_bytes || (need && !ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_sparse_attn: workspace too small");
     CUtensorMap tkv;
-    if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(B) * Lk,
+    if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(kv_rows),
                          static_cast<uint64_t>(k_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSA_ERR_CUDA, "tensor map for the latent cache failed");
     MlaParams p{};
@@ -822,7 +870,11 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
                           : nullptr;
     p.err = device_error_word();
     if (!p.err) return set_error(DSA_ERR_CUDA, "cannot resolve the device error word");
+    p.cu_q = vl ? vl->cu_q : nullptr;
+    p.cu_k = vl ? vl->cu_k : nullptr;
+    p.sp = vl ? vl->sp : nullptr;
     p.B = B; p.Lq = Lq; p.Lk = Lk; p.start_pos = start_pos; p.k = k;
+    p.rows = static_cast<int>(rows);
     p.S = sp.S; p.cps = sp.cps;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(mla_sparse_attn_kernel), kMlaSmem);
@@ -850,7 +902,8 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
                                stream, reinterpret_cast<const __nv_bfloat16*>(q),
                                reinterpret_cast<const __nv_bfloat16*>(kbuf), k_row_stride,
                                reinterpret_cast<const __nv_bfloat16*>(vbuf), v_row_stride, idx, B, Lq, Lk,
-                               start_pos, n_h, D_qk, D_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse);
+                               start_pos, n_h, D_qk, D_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse,
+                               vl ? vl->cu_q : nullptr, vl ? vl->cu_k : nullptr, vl ? vl->sp : nullptr);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("simt attention launch: ") + cudaGetErrorString(e));
     return DSA_OK;

@@ -24,7 +24,14 @@ EXPORTS = ["dsa_last_error", "dsa_indexer_topk_workspace", "dsa_indexer_topk",
            "indexcache_forward", "dsa_indexer_launch_count", "dsa_check_device_errors",
            "dsa_indexer_topk_noalloc", "dsa_selftest_wait_timeout", "dsa_check_indices",
            "dsa_dense_weights", "dsa_topk_rows", "dsa_index_overlap", "dsa_captured_mass",
-           "dsa_csa_indexer_topk_workspace", "dsa_csa_indexer_topk", "dsa_csa_sparse_attn"]
+           "dsa_csa_indexer_topk_workspace", "dsa_csa_indexer_topk", "dsa_csa_sparse_attn",
+           "dsa_indexer_topk_varlen_workspace", "dsa_indexer_topk_varlen",
+           "dsa_sparse_attn_varlen_workspace", "dsa_sparse_attn_varlen",
+           "indexcache_forward_varlen_workspace", "indexcache_forward_varlen", "dsa_check_varlen",
+           "dsa_indexer_topk_lowprec_workspace", "dsa_indexer_topk_lowprec", "dsa_mx_quantize"]
+
+DSA_FMT_E4M3, DSA_FMT_E2M1 = 0, 1
+FORMATS = {"e4m3": DSA_FMT_E4M3, "e2m1": DSA_FMT_E2M1}
 
 
 class DSAError(RuntimeError):
@@ -45,6 +52,12 @@ class LayerIO(ctypes.Structure):
     _fields_ = [("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("q", ctypes.c_void_p), ("kbuf", ctypes.c_void_p), ("vbuf", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+
+
+class Varlen(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("cu_q", ctypes.c_void_p), ("cu_k", ctypes.c_void_p),
+                ("start_pos", ctypes.c_void_p), ("total_q", ctypes.c_int), ("total_k", ctypes.c_int),
+                ("max_Lq", ctypes.c_int), ("max_Lk", ctypes.c_int)]
 
 
 _lib = None
@@ -98,6 +111,28 @@ def lib():
         L.dsa_csa_sparse_attn.argtypes = [P, P, I64, P, I, I, I, I, I, I, I, I, I, F32, P, P, P,
                                           SZ, P]
         L.dsa_csa_sparse_attn.restype = I
+        VP = ctypes.POINTER(Varlen)
+        L.dsa_indexer_topk_varlen_workspace.argtypes = [VP, I, I, I]
+        L.dsa_indexer_topk_varlen_workspace.restype = SZ
+        L.dsa_indexer_topk_varlen.argtypes = [P, P, P, VP, I, I, I, P, P, SZ, P]
+        L.dsa_indexer_topk_varlen.restype = I
+        L.dsa_sparse_attn_varlen_workspace.argtypes = [VP, I, I, I]
+        L.dsa_sparse_attn_varlen_workspace.restype = SZ
+        L.dsa_sparse_attn_varlen.argtypes = [P, P, I64, P, I64, P, VP, I, I, I, I, F32, P, P, P, SZ, P]
+        L.dsa_sparse_attn_varlen.restype = I
+        L.indexcache_forward_varlen_workspace.argtypes = [ctypes.POINTER(Dims), VP]
+        L.indexcache_forward_varlen_workspace.restype = SZ
+        L.indexcache_forward_varlen.argtypes = [ctypes.c_char_p, I, ctypes.POINTER(LayerIO),
+                                                ctypes.POINTER(Dims), VP, P, P, SZ, P]
+        L.indexcache_forward_varlen.restype = I
+        L.dsa_check_varlen.argtypes = [VP, P, P]
+        L.dsa_check_varlen.restype = I
+        L.dsa_indexer_topk_lowprec_workspace.argtypes = [I] * 8
+        L.dsa_indexer_topk_lowprec_workspace.restype = SZ
+        L.dsa_indexer_topk_lowprec.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, P, SZ, P]
+        L.dsa_indexer_topk_lowprec.restype = I
+        L.dsa_mx_quantize.argtypes = [P, I64, I, I, P, P, P]
+        L.dsa_mx_quantize.restype = I
         _lib = L
     return _lib
 
@@ -368,3 +403,153 @@ def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
     abandoned after `limit_cycles`); the next check_device_errors() raises
     DSA_ERR_TIMEOUT."""
     _check(lib().dsa_selftest_wait_timeout(int(limit_cycles), stream if stream is not None else _stream()))
+
+
+# --------------------------------------------------------------------------
+# Variable-length batches (packed rows; see dsa_varlen in include/dsa.h)
+class VarlenBatch:
+    """A variable-length batch: the device offset arrays and the host sizes
+    of ``dsa_varlen``.  Keeps the device arrays alive with the descriptor."""
+
+    def __init__(self, q_lens, k_lens, start_pos, device="cuda"):
+        import torch
+        q_lens, k_lens, start_pos = list(map(int, q_lens)), list(map(int, k_lens)), list(map(int, start_pos))
+        if not (len(q_lens) == len(k_lens) == len(start_pos) >= 1):
+            raise ValueError("q_lens, k_lens and start_pos need one entry per sequence")
+        cu_q, cu_k = [0], [0]
+        for a, b in zip(q_lens, k_lens):
+            cu_q.append(cu_q[-1] + a)
+            cu_k.append(cu_k[-1] + b)
+        self.q_lens, self.k_lens, self.start_pos_list = q_lens, k_lens, start_pos
+        self.cu_q_list, self.cu_k_list = cu_q, cu_k
+        self.cu_q = torch.tensor(cu_q, dtype=torch.int32, device=device)
+        self.cu_k = torch.tensor(cu_k, dtype=torch.int32, device=device)
+        self.start_pos = torch.tensor(start_pos, dtype=torch.int32, device=device)
+        self.desc = Varlen(B=len(q_lens), cu_q=self.cu_q.data_ptr(), cu_k=self.cu_k.data_ptr(),
+                           start_pos=self.start_pos.data_ptr(), total_q=cu_q[-1], total_k=cu_k[-1],
+                           max_Lq=max(max(q_lens), 1), max_Lk=max(max(k_lens), 1))
+
+    @property
+    def B(self):
+        return self.desc.B
+
+    @property
+    def total_q(self):
+        return self.desc.total_q
+
+    @property
+    def total_k(self):
+        return self.desc.total_k
+
+
+def indexer_topk_varlen(q_idx, k_idx, w, k: int, vb: VarlenBatch, *, out=None, ws=None):
+    """Lightning indexer + top-k per sequence of a packed batch: q_idx
+    [total_q, H, d] bf16, k_idx [total_k, d] bf16, w [total_q, H] f32 ->
+    idx [total_q, k] int32."""
+    import torch
+    tq, H, d = q_idx.shape
+    _need(q_idx, torch.bfloat16, (vb.total_q, H, d), "q_idx")
+    _need(k_idx, torch.bfloat16, (vb.total_k, d), "k_idx")
+    _need(w, torch.float32, (vb.total_q, H), "w")
+    if out is None:
+        out = torch.empty((vb.total_q, k), dtype=torch.int32, device=q_idx.device)
+    _need(out, torch.int32, (vb.total_q, k), "out")
+    need = int(lib().dsa_indexer_topk_varlen_workspace(ctypes.byref(vb.desc), H, d, k))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_idx.device)
+    _check(lib().dsa_indexer_topk_varlen(_ptr(q_idx), _ptr(k_idx), _ptr(w), ctypes.byref(vb.desc), H, d, k,
+                                         _ptr(out), _ptr(ws), ws.numel(), _stream(q_idx)))
+    return out
+
+
+def sparse_attn_varlen(q, kbuf, vbuf, idx, scale: float, vb: VarlenBatch, *, D_v: int, out=None, lse=None,
+                       ws=None):
+    """Sparse core attention per sequence of a packed batch: q [total_q, n_h,
+    D_qk] bf16, kbuf/vbuf [total_k, C] bf16 rows, idx [total_q, k] int32 ->
+    out [total_q, n_h, D_v] bf16 (and lse [total_q, n_h] f32 if given)."""
+    import torch
+    tq, n_h, D_qk = q.shape
+    k = idx.shape[1]
+    _need(q, torch.bfloat16, (vb.total_q, n_h, D_qk), "q")
+    _need(kbuf, torch.bfloat16, name="kbuf")
+    _need(vbuf, torch.bfloat16, name="vbuf")
+    if kbuf.shape[0] != vb.total_k or vbuf.shape[0] != vb.total_k:
+        raise ValueError("kbuf and vbuf need total_k rows")
+    _need(idx, torch.int32, (vb.total_q, k), "idx")
+    if out is None:
+        out = torch.empty((vb.total_q, n_h, D_v), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, (vb.total_q, n_h, D_v), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (vb.total_q, n_h), "lse")
+    need = int(lib().dsa_sparse_attn_varlen_workspace(ctypes.byref(vb.desc), n_h, D_v, k))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().dsa_sparse_attn_varlen(_ptr(q), _ptr(kbuf), kbuf.shape[1], _ptr(vbuf), vbuf.shape[1], _ptr(idx),
+                                        ctypes.byref(vb.desc), n_h, D_qk, D_v, k, float(scale), _ptr(out),
+                                        _ptr(lse), _ptr(ws), ws.numel(), _stream(q)))
+    return out
+
+
+def indexcache_forward_varlen(pattern: str, layers, dims: Dims, vb: VarlenBatch, idx_cache, ws=None):
+    """The F/S layer loop over a packed batch; ``layers`` as for
+    indexcache_forward with packed per-layer tensors, idx_cache [total_q, k]."""
+    import torch
+    n = len(layers)
+    arr = (LayerIO * max(n, 1))()
+    for i, L in enumerate(layers):
+        arr[i] = LayerIO(*[(L[f].data_ptr() if L.get(f) is not None else None) for f in
+                           ("q_idx", "k_idx", "w", "q", "kbuf", "vbuf", "out", "lse")])
+    need = int(lib().indexcache_forward_varlen_workspace(ctypes.byref(dims), ctypes.byref(vb.desc)))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=idx_cache.device)
+    _check(lib().indexcache_forward_varlen(pattern.encode(), n, arr, ctypes.byref(dims), ctypes.byref(vb.desc),
+                                           _ptr(idx_cache), _ptr(ws), ws.numel(), _stream(idx_cache)))
+    return idx_cache
+
+
+def check_varlen(vb: VarlenBatch) -> int:
+    """Number of sequences of the batch that break the dsa_varlen contract
+    (checked on the device).  Synchronises the current stream."""
+    import torch
+    bad = torch.empty(1, dtype=torch.int32, device=vb.cu_q.device)
+    _check(lib().dsa_check_varlen(ctypes.byref(vb.desc), _ptr(bad), _stream(vb.cu_q)))
+    return int(bad.item())
+
+
+# --------------------------------------------------------------------------
+# Low-precision selector ([IDX] §5.4; MX E4M3 / E2M1 operands, bf16 scores)
+def indexer_topk_lowprec_workspace(B, Lq, Lk, start_pos, H_I, d_I, k, fmt: str) -> int:
+    return int(lib().dsa_indexer_topk_lowprec_workspace(B, Lq, Lk, start_pos, H_I, d_I, k, FORMATS[fmt]))
+
+
+def indexer_topk_lowprec(q_idx, k_idx, w, k: int, *, fmt: str, start_pos: int = 0, out=None, ws=None):
+    """Low-precision selector: q_idx [B,Lq,64,128] bf16, k_idx [B,Lk,128]
+    bf16, w [B,Lq,64] f32 quantised to MX ``fmt`` ("e4m3" or "e2m1") inside
+    the call -> idx [B,Lq,k] int32 (bf16 scores, ascending, -1 padded)."""
+    import torch
+    B, Lq, H, d = q_idx.shape
+    Lk = k_idx.shape[1]
+    _need(q_idx, torch.bfloat16, name="q_idx")
+    _need(k_idx, torch.bfloat16, (B, Lk, d), "k_idx")
+    _need(w, torch.float32, (B, Lq, H), "w")
+    if out is None:
+        out = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device)
+    _need(out, torch.int32, (B, Lq, k), "out")
+    need = indexer_topk_lowprec_workspace(B, Lq, Lk, start_pos, H, d, k, fmt)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_idx.device)
+    _check(lib().dsa_indexer_topk_lowprec(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Lq, Lk, start_pos, H, d, k,
+                                          FORMATS[fmt], _ptr(out), _ptr(ws), ws.numel(), _stream(q_idx)))
+    return out
+
+
+def mx_quantize(x, fmt: str):
+    """MX quantisation of bf16 rows x [..., 128] -> (codes uint8 [rows, 128],
+    scales uint8 [rows, 4]); see dsa_mx_quantize."""
+    import torch
+    _need(x, torch.bfloat16, name="x")
+    rows = x.numel() // x.shape[-1]
+    codes = torch.empty((rows, x.shape[-1]), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, x.shape[-1] // 32), dtype=torch.uint8, device=x.device)
+    _check(lib().dsa_mx_quantize(_ptr(x), rows, x.shape[-1], FORMATS[fmt], _ptr(codes), _ptr(scales), _stream(x)))
+    return codes, scales

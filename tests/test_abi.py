@@ -169,3 +169,77 @@ def test_csa_entry_points_validated_on_host():
                                    fake, None, fake, 0, None) == E
     assert lib.dsa_csa_sparse_attn(fake, fake, 500, fake, 1, 8, 2, 0, 4, 128, 576, 512, 8, 1.0,
                                    fake, None, fake, 0, None) == E
+
+
+def _varlen(B=2, total_q=10, total_k=20, max_Lq=6, max_Lk=12, arrays=True):
+    fake = 1 << 20  # never dereferenced on the host
+    return dsa.Varlen(B=B, cu_q=fake if arrays else None, cu_k=fake if arrays else None,
+                      start_pos=fake if arrays else None, total_q=total_q, total_k=total_k,
+                      max_Lq=max_Lq, max_Lk=max_Lk)
+
+
+def test_varlen_entry_points_validated_on_host():
+    lib = dsa.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    E = dsa.DSA_ERR_INVALID_ARG
+    good = _varlen()
+    for bad in (None, _varlen(arrays=False), _varlen(B=0), _varlen(max_Lq=11), _varlen(max_Lk=21),
+                _varlen(total_q=0)):
+        ref = ctypes.byref(bad) if bad is not None else None
+        assert lib.dsa_indexer_topk_varlen(fake, fake, fake, ref, 64, 128, 8, fake, fake, 1 << 30, None) == E
+        assert lib.dsa_sparse_attn_varlen(fake, fake, 576, fake, 576, fake, ref, 128, 576, 512, 8, 1.0, fake,
+                                          None, fake, 1 << 30, None) == E
+        assert lib.dsa_check_varlen(ref, fake, None) == E
+        assert lib.dsa_indexer_topk_varlen_workspace(ref, 64, 128, 8) == 0
+    # misaligned offset array
+    mis = _varlen()
+    mis.cu_q = (1 << 20) + 2
+    assert lib.dsa_check_varlen(ctypes.byref(mis), fake, None) == E
+    g = ctypes.byref(good)
+    # the per-sequence limits of the uniform indexer apply
+    assert lib.dsa_indexer_topk_varlen(fake, fake, fake, g, 12, 128, 8, fake, fake, 1 << 30,
+                                       None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_topk_varlen(fake, fake, fake, g, 64, 128, 8, None, fake, 1 << 30, None) == E
+    assert lib.dsa_indexer_topk_varlen(fake, fake, fake, g, 64, 128, 8, fake, fake, 16,
+                                       None) == dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_indexer_topk_varlen_workspace(g, 64, 128, 8) > 0
+    # attention: row stride shorter than the row
+    assert lib.dsa_sparse_attn_varlen(fake, fake, 64, fake, 576, fake, g, 128, 576, 512, 8, 1.0, fake, None, fake,
+                                      1 << 30, None) == E
+    # layer loop: the pattern rule holds for varlen batches too
+    d = dsa.Dims(B=1, Lq=8, Lk=8, start_pos=0, H_I=64, d_I=128, k=4, n_h=128, D_qk=576, D_v=512,
+                 scale=1.0, k_row_stride=576, v_row_stride=576)
+    arr = (dsa.LayerIO * 2)()
+    assert lib.indexcache_forward_varlen(b"SF", 2, arr, ctypes.byref(d), g, fake, fake, 1 << 30,
+                                         None) == dsa.DSA_ERR_BAD_PATTERN
+    assert lib.indexcache_forward_varlen(b"FS", 2, arr, ctypes.byref(d), g, fake, fake, 1 << 30, None) == E
+
+
+def test_varlen_decode_batches_take_the_decode_workspace():
+    # one query row per sequence (max_Lq = 1, total_q = B): the decode kernels
+    # keep one row of score keys per sequence, sized by the longest cache
+    lib = dsa.lib()
+    dec = _varlen(B=8, total_q=8, total_k=8 * 200000, max_Lq=1, max_Lk=200000)
+    ws = lib.dsa_indexer_topk_varlen_workspace(ctypes.byref(dec), 64, 128, 2048)
+    assert ws == lib.dsa_indexer_topk_workspace(8, 1, 200000, 200000, 64, 128, 2048)
+
+
+def test_lowprec_entry_points_validated_on_host():
+    lib = dsa.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    E, U = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
+    # (q, k, w, B, Lq, Lk, start, H, d, k, fmt, idx, ws, ws_bytes, stream)
+    assert lib.dsa_indexer_topk_lowprec(None, fake, fake, 1, 8, 8, 0, 64, 128, 4, 0, fake, fake, 1 << 30, None) == E
+    assert lib.dsa_indexer_topk_lowprec(fake, fake, fake, 1, 8, 8, 0, 64, 128, 4, 7, fake, fake, 1 << 30, None) == E
+    assert lib.dsa_indexer_topk_lowprec(fake, fake, fake, 1, 8, 8, 0, 32, 128, 4, 0, fake, fake, 1 << 30, None) == U
+    assert lib.dsa_indexer_topk_lowprec(fake, fake, fake, 1, 8, 8, 0, 64, 64, 4, 1, fake, fake, 1 << 30, None) == U
+    assert lib.dsa_indexer_topk_lowprec(fake, fake, fake, 1, 8, 8, 5, 64, 128, 4, 0, fake, fake, 1 << 30, None) == E
+    assert lib.dsa_indexer_topk_lowprec(fake, fake, fake, 1, 8, 8, 0, 64, 128, 4, 0, fake, fake, 16,
+                                        None) == dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_indexer_topk_lowprec_workspace(1, 8, 8, 0, 64, 128, 4, 9) == 0
+    assert lib.dsa_indexer_topk_lowprec_workspace(1, 8, 8, 0, 64, 128, 4, 1) > 8 * 64 * 128 + 8 * 128
+    # (x, rows, cols, fmt, codes, scales, stream)
+    assert lib.dsa_mx_quantize(fake, 0, 128, 0, fake, fake, None) == E
+    assert lib.dsa_mx_quantize(fake, 4, 96, 0, fake, fake, None) == U
+    assert lib.dsa_mx_quantize(fake, 4, 128, 3, fake, fake, None) == E
+    assert lib.dsa_mx_quantize(None, 4, 128, 0, fake, fake, None) == E

@@ -934,8 +934,10 @@ def kernel_case(name, seq, reps):
     from sparse_attention_13_b200 import dsa, synth
     dev = torch.device("cuda", 0)
     bf = torch.bfloat16
-    if name in ("indexer", "decode_idx"):
-        B, Lq, Lk, sp = (1, seq, seq, 0) if name == "indexer" else (8, 1, 200000, 200000)
+    if name in ("indexer", "decode_idx", "indexer_tail"):
+        # indexer_tail: the last `seq` query rows of a 200,000-token prefill
+        B, Lq, Lk, sp = {"indexer": (1, seq, seq, 0), "decode_idx": (8, 1, 200000, 200000),
+                         "indexer_tail": (1, seq, 200000, 200000 - seq)}[name]
         q = torch.empty((B, Lq, 64, 128), dtype=bf, device=dev)
         kk = torch.empty((B, Lk, 128), dtype=bf, device=dev)
         w = torch.empty((B, Lq, 64), dtype=torch.float32, device=dev)
@@ -945,8 +947,11 @@ def kernel_case(name, seq, reps):
         out = torch.empty((B, Lq, 2048), dtype=torch.int32, device=dev)
         ws = torch.empty(dsa.indexer_topk_workspace(B, Lq, Lk, sp, 64, 128, 2048), dtype=torch.uint8, device=dev)
         run = lambda: dsa.indexer_topk(q, kk, w, 2048, start_pos=sp, out=out, ws=ws)
-    elif name in ("attn", "decode_attn"):
-        B, Lq, Lk, sp = (1, seq, seq, 0) if name == "attn" else (8, 1, 200000, 200000)
+    elif name in ("attn", "decode_attn", "attn_tail"):
+        # attn_tail: the last `seq` rows of a 200,000-token prefill against the
+        # full latent cache (the long-context gather regime on a few GB)
+        B, Lq, Lk, sp = {"attn": (1, seq, seq, 0), "decode_attn": (8, 1, 200000, 200000),
+                         "attn_tail": (1, seq, 200000, 200000 - seq)}[name]
         q = torch.empty((B, Lq, 128, 576), dtype=bf, device=dev)
         kv = torch.empty((B, Lk, 576), dtype=bf, device=dev)
         synth.fill_cuda(q, SEED, synth.Q, synth.NORMAL, 0, sigma=0.5)
@@ -1198,7 +1203,7 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="override the prefill length (testing)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default="",
-                    help="profiling: indexer|attn|decode_idx|decode_attn|decode_step; "
+                    help="profiling: indexer|indexer_tail|attn|attn_tail|decode_idx|decode_attn|decode_step; "
                          "quality runs the selection-quality tools, csa one CSA-style layer, "
                          "lowprec the low-precision selector's recall and times")
     ap.add_argument("--reps", type=int, default=2)

@@ -245,9 +245,11 @@ dsa_status dsa_indexer_topk_lowprec(const dsa_bf16 *q_idx, const dsa_bf16 *k_idx
                                     size_t ws_bytes, void *stream);
 
 /* MX quantisation of bf16 rows (the rule above): x [rows, cols] bf16 ->
- * codes [rows, cols] (one byte per element: an E4M3 code, or an E2M1 code in
- * bits 2..5 of its byte) and scales [rows, cols / 32] (the block exponent E
- * as E + 127).  Supported: cols = 128. */
+ * codes [rows, cols] bytes and scales [rows, cols / 32] (the block exponent
+ * E as E + 127).  E4M3: one code per byte.  E2M1: element 16 g + j of a row
+ * sits in byte 16 g + j / 2 (the low nibble for even j), and bytes
+ * 16 g + 8 .. 16 g + 15 are zero (the layout block-scaled tensor-core
+ * products read 4-bit operands in).  Supported: cols = 128. */
 dsa_status dsa_mx_quantize(const dsa_bf16 *x, int64_t rows, int cols, int fmt,
                            uint8_t *codes, uint8_t *scales, void *stream);
 

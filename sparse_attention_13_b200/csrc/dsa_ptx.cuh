@@ -103,17 +103,15 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
-// Asynchronous 16-byte store into a (possibly remote) CTA's shared memory in
-// the cluster; the store signals complete_tx(16) on the mbarrier at
-// bar_cluster, which must sit in the same CTA as the destination.  No memory
-// clobber: the issuing thread never reads the destination, and volatile asm
-// statements keep their order relative to the waits and arrivals around it.
-__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint32_t a, uint32_t b, uint32_t c,
-                                            uint32_t d, uint32_t bar_cluster) {
+// Bulk DMA from this CTA's shared memory into a peer CTA's shared memory,
+// signalling complete_tx(bytes) on the peer's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_smem,
+                                                  uint32_t bytes, uint32_t bar_cluster) {
   asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-          dst_cluster),
-      "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster));
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst_cluster),
+      "r"(src_smem), "r"(bytes), "r"(bar_cluster)
+      : "memory");
 }
 // One contiguous global -> shared copy by the bulk-copy engine, completing
 // on a CTA-local mbarrier (both addresses 16-byte aligned, size a multiple of
@@ -124,6 +122,13 @@ __device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the source of every committed bulk copy has been read.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -12,8 +12,10 @@
 // mx_quantize_kernel  one warp per row of 128 bf16 elements (4 blocks): block
 //     maxima by warp shuffles, the exponent from the bit pattern of the
 //     maximum, conversions by the hardware's round-to-nearest-even,
-//     saturating cvt.  Codes are one byte per element (E2M1 codes in the
-//     layout the block-scaled MMA reads from 8-bit containers).  Scales go
+//     saturating cvt.  E4M3 codes are one byte per element; E2M1 codes are
+//     packed two per byte, 16 codes in the first half of each 16-byte slot
+//     (the layout the block-scaled MMA reads sub-byte operands in), so a row
+//     takes 128 bytes either way.  Scales go
 //     either row-major ([rows][4]) or grouped by 128 rows in the layout the
 //     TMEM copy of the MMA kernel reads.
 // The selector itself is the fused indexer + top-k kernel of indexer_topk.cu
@@ -33,9 +35,6 @@ namespace {
 
 constexpr int kCols = 128;          // elements per row (d_I)
 constexpr int kQuantThreads = 256;  // 8 rows per block
-// Bit position of an E2M1 code inside its 8-bit container, as the
-// block-scaled MMA of kind::mxf8f6f4 reads it.
-constexpr int kE2M1Shift = 2;
 
 template <int FMT>  // 0: E4M3, 1: E2M1
 __global__ void __launch_bounds__(kQuantThreads)
@@ -78,12 +77,22 @@ mx_quantize_kernel(const __nv_bfloat16* __restrict__ x, int B, long long rows_pe
           __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v[2], -e), ldexpf(v[3], -e)), __NV_SATFINITE, __NV_E4M3);
       packed = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
     } else {
+      // two codes per byte, the even element in the low nibble
       const __nv_fp4x2_storage_t lo =
           __nv_cvt_float2_to_fp4x2(make_float2(ldexpf(v[0], -e), ldexpf(v[1], -e)), __NV_E2M1, cudaRoundNearest);
       const __nv_fp4x2_storage_t hi =
           __nv_cvt_float2_to_fp4x2(make_float2(ldexpf(v[2], -e), ldexpf(v[3], -e)), __NV_E2M1, cudaRoundNearest);
-      const uint32_t c0 = lo & 0xF, c1 = (lo >> 4) & 0xF, c2 = hi & 0xF, c3 = (hi >> 4) & 0xF;
-      packed = (c0 << kE2M1Shift) | (c1 << (8 + kE2M1Shift)) | (c2 << (16 + kE2M1Shift)) | (c3 << (24 + kE2M1Shift));
+      const uint32_t mine = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 8);
+      // The block-scaled MMA reads sub-byte operands as 16 codes packed in
+      // the first 8 bytes of each 16-byte slot (the rest zero): word l of
+      // the row is slot l / 4, quarter q = l % 4; quarters 0 and 1 hold the
+      // slot's codes 0-7 and 8-15, i.e. the 16-bit pieces of lanes
+      // 4 (l / 4) + 2 q and the next one.
+      const int q = lane & 3;
+      const int src = (lane & ~3) + 2 * (q & 1);
+      const uint32_t a = __shfl_sync(0xffffffffu, mine, src);
+      const uint32_t b2 = __shfl_sync(0xffffffffu, mine, src + 1);
+      packed = q < 2 ? (a | (b2 << 16)) : 0u;
     }
     reinterpret_cast<uint32_t*>(codes + row * kCols)[lane] = packed;
     if ((lane & 7) == 0) sfp[lane >> 3] = static_cast<uint8_t>(min(max(e + 127, 0), 254));

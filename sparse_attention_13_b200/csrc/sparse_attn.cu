@@ -19,12 +19,13 @@
 //                    a double-buffered S tile, then, one chunk behind,
 //                    O_c += P V_c with P read from TMEM and V_c the gathered
 //                    slabs 0..3 read as an MN-major B operand;
-//     4 sender warps (thread = head) read S_c as soon as QK completes and
-//                    store it, fp32, straight into the peer's shared memory
-//                    with asynchronous remote stores that count their bytes
-//                    on the peer's mbarrier; they also load the next row's
-//                    query into TMEM as soon as the last QK of the current row
-//                    has completed;
+//     4 sender warps (thread = head) read S_c as soon as QK completes,
+//                    stage it, fp32, in shared memory and ship it to the peer
+//                    with one bulk copy into the peer's shared memory
+//                    (tx-counted on its mbarrier; the peer frees the tile as
+//                    soon as its softmax has read it); they also load the
+//                    next row's query into TMEM as soon as the last QK of the
+//                    current row has completed;
 //     8 softmax warps (thread = head = TMEM lane x half of the chunk) add the
 //                    peer's partial (S = S_0 + S_1, identical in both CTAs as
 //                    fp32 addition commutes), mask padded rows (fully valid
@@ -157,6 +158,7 @@ constexpr int kMaxSlabs = 5;                   // CTA0: columns 0..255, CTA1: 25
 constexpr int kStageBytes = kMaxSlabs * kSlabBytes;
 constexpr int kStages = 3;
 constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile, fp32
+constexpr int kXHalf = kXBytes / 2;            // one half: 32 columns of 128 heads, [head][32] fp32
 constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, bf16
 // TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64; P(c) overwrites
 // the first 32 columns of S(c) as bf16 pairs) | Q (bf16 pairs, 128)
@@ -175,7 +177,7 @@ struct MlaBars {
   uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
   uint64_t o_full, o_free, q_full;
   uint64_t q0_full;  // first item: Q loaded by the sender and softmax warps together
-  uint64_t x_full[2], x_free[2];
+  uint64_t x_full, x_free;  // the peer's partial tile landed / consumed
   unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
   float lsum[1][2][kNH];                        // [half][head] final sums
@@ -183,7 +185,8 @@ struct MlaBars {
   int abort_flag;
 };
 
-// shared memory: gather ring | peer partials X_in[2] (fp32) | Q rope
+// shared memory: gather ring | the peer's partials X_in (fp32) | this CTA's
+// partials staged for the copy X_out | Q rope
 constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kQRopeBytes +
                          static_cast<int>(sizeof(MlaBars)) + 64;
 
@@ -231,8 +234,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* kv_smem = smem;
-  uint8_t* xin_smem = kv_smem + kStages * kStageBytes;   // X_in[2]: the peer's partials
-  uint8_t* qrope_smem = xin_smem + 2 * kXBytes;          // CTA1: Q[:, 512:576]
+  uint8_t* xin_smem = kv_smem + kStages * kStageBytes;   // X_in[half]: the peer's partials
+  uint8_t* xout_smem = xin_smem + kXBytes;               // X_out[half]: this CTA's, staged
+  uint8_t* qrope_smem = xout_smem + kXBytes;             // CTA1: Q[:, 512:576]
   MlaBars* bb = reinterpret_cast<MlaBars*>(qrope_smem + kQRopeBytes);
   volatile int* abort_flag = &bb->abort_flag;
 
@@ -258,9 +262,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       mbar_init(&bb->s_read[b], kSendWarps);
       mbar_init(&bb->p_full[b], kSoftWarps);
       mbar_init(&bb->pv_done[b], 1);
-      mbar_init(&bb->x_full[b], 1);
-      mbar_init(&bb->x_free[b], kSoftWarps);
     }
+    // X_in: the peer's bulk copy completes the phase; the phase of chunk 0 is
+    // armed here, the next one by the softmax as it consumes a chunk
+    mbar_init(&bb->x_full, 1);
+    mbar_init(&bb->x_free, kSoftWarps);
+    mbar_arrive_expect_tx(&bb->x_full, kXBytes);
     mbar_init(&bb->o_full, 1);
     mbar_init(&bb->o_free, kSoftWarps);
     mbar_init(&bb->q_full, kSendWarps);
@@ -414,8 +421,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int stid = threadIdx.x - kSendWarp0 * 32;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const uint32_t xin_remote = mapa_shared(smem_u32(xin_smem), peer);
-    // x_full[0] and x_full[1] are adjacent: the peer's x_full[sb] is at + 8 sb
-    const uint32_t xfull_remote = mapa_shared(smem_u32(&bb->x_full[0]), peer);
+    const uint32_t xfull_remote = mapa_shared(smem_u32(&bb->x_full), peer);
     // A failed (timed-out) wait only clears `ok`; the sender warps leave their
     // loops together, at the next named barrier, so none is left waiting there.
     uint32_t g = 0, it_n = 0;
@@ -468,37 +474,45 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         if (c == c_pf && nq != nullptr)
           for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag));
-        // the peer's X_in[sb] is free once its softmax has consumed chunk g-2
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_free[sb], ((g >> 1) & 1) ^ 1, abort_flag));
         tc_fence_after();
+        // X_out is free once the previous chunk's copy has read it
+        if (stid == 0) bulk_wait_read_all();
+        ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
         if (ok) {
-          // this CTA's X_in[sb] receives the peer's partial of chunk g: one
-          // arrival plus its bytes complete the phase
-          if (stid == 0) mbar_arrive_expect_tx(&bb->x_full[sb], kXBytes);
-          // row h of the peer's tile, 16-byte pieces XOR-swizzled by h & 7 so
-          // that the peer's per-head reads are free of bank conflicts: piece j
-          // of the row sits at byte offset off ^ (j << 4) of X_in (bits 4..7 of
-          // off are h & 7 and zero above, for j < 16)
-          const uint32_t off = sb * kXBytes + h * 256 + ((h & 7) << 4);
-#pragma unroll
-          for (int hv = 0; hv < 4; ++hv) {
-            uint32_t v[16];
-            tmem_ld32<16>(t_lane + kSCol + sb * 64 + hv * 16, v);
+          // row h of each 32-column half: 16-byte pieces XOR-swizzled by
+          // h & 7, so that the peer's per-head reads are free of bank conflicts
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld32<32>(t_lane + kSCol + sb * 64 + half * 32, v);
             tmem_ld_wait();
+            uint8_t* xo = xout_smem + half * kXHalf + h * 128;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              st_async_v4(xin_remote + (off ^ ((4 * hv + j) << 4)), v[4 * j], v[4 * j + 1], v[4 * j + 2],
-                          v[4 * j + 3], xfull_remote + 8 * sb);
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(xo + ((j ^ (h & 7)) << 4)) =
+                  make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(&bb->s_read[sb]);
+        fence_proxy_async_smem();
+        named_bar_sync(kSendBar + 1, kSendWarps * 32);
+        if (stid == 0 && ok) {
+          // the peer's X_in is free once its softmax has consumed chunk g-1
+          if (mbar_wait_cluster(&bb->x_free, (g & 1) ^ 1, abort_flag)) {
+            bulk_copy_to_peer(xin_remote, smem_u32(xout_smem), kXBytes, xfull_remote);
+            bulk_commit_group();
+          } else {
+            ok = false;  // the abort flag is raised; the next barrier ends the loop
+          }
+        }
       }
       ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
       if (!ok) break;
       ++it_n;
     }
+    if (stid == 0) bulk_wait_read_all();  // the last copy has read the staging buffer
   } else {
     // ------------------------------------------------------------ softmax
     // thread = (head h = TMEM lane, half hf of the chunk's 64 columns)
@@ -506,8 +520,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int h = qd * 32 + lane;
     const int pair_bar = kPairBarBase + qd;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const uint32_t xfree_remote[2] = {mapa_shared(smem_u32(&bb->x_free[0]), peer),
-                                      mapa_shared(smem_u32(&bb->x_free[1]), peer)};
+    const uint32_t xfree_remote = mapa_shared(smem_u32(&bb->x_free), peer);
     // A failed (timed-out) wait only clears `ok`; the two warps of a head pair
     // leave their loops together at the next pair barrier.
     uint32_t g = 0, it_n = 0;
@@ -574,18 +587,23 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
         }
         // + the peer's partial scores of the same columns (fp32)
-        if (ok) ok = mbar_wait_cluster(&bb->x_full[sb], (g >> 1) & 1, abort_flag);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_full, g & 1, abort_flag));
         if (ok) {
-          const uint8_t* xr = xin_smem + sb * kXBytes + h * 256;
+          const uint8_t* xr = xin_smem + hf * kXHalf + h * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 o = *reinterpret_cast<const float4*>(xr + (((hf * 8 + j) ^ (h & 7)) << 4));
+            const float4 o = *reinterpret_cast<const float4*>(xr + ((j ^ (h & 7)) << 4));
             s[4 * j] += o.x;
             s[4 * j + 1] += o.y;
             s[4 * j + 2] += o.z;
             s[4 * j + 3] += o.w;
           }
         }
+        // X_in is consumed (the additions above used every loaded value):
+        // arm the phase of the next chunk, then let the peer send it
+        __syncwarp();
+        if (threadIdx.x == 0 && ok) mbar_arrive_expect_tx(&bb->x_full, kXBytes);
+        if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote);
         // mask, scale, chunk max (combined with the other half of the head)
         if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
         float lmax = -INFINITY;
@@ -663,11 +681,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && ok) {
-          mbar_arrive(&bb->p_full[sb]);
-          // X_in[sb] was consumed above: the peer may send chunk g+2 into it
-          mbar_arrive_remote_relaxed(xfree_remote[sb]);
-        }
+        if (lane == 0 && ok) mbar_arrive(&bb->p_full[sb]);
       }
       // combine the two halves' sums
       bb->lsum[0][hf][h] = l_run;

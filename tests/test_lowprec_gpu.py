@@ -34,7 +34,11 @@ def _decode_e4m3(c):
 
 
 def _decode_e2m1(byte):
-    c = (byte.astype(np.int64) >> 2) & 15   # code in bits 2..5 of its byte
+    # 16 codes per 16-byte slot, packed in its first 8 bytes, low nibble first
+    rows, cols = byte.shape
+    slot = byte.astype(np.int64).reshape(rows, cols // 16, 16)
+    assert np.all(slot[:, :, 8:] == 0)
+    c = np.stack([slot[:, :, :8] & 15, slot[:, :, :8] >> 4], axis=-1).reshape(rows, cols)
     s = np.where(c & 8, -1.0, 1.0)
     e = (c >> 1) & 3
     m = c & 1

@@ -159,25 +159,30 @@ constexpr int kStageBytes = kMaxSlabs * kSlabBytes;
 constexpr int kStages = 3;
 constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile, fp32
 constexpr int kXHalf = kXBytes / 2;            // one half: 32 columns of 128 heads, [head][32] fp32
+constexpr int kPBytes = kNH * kChunk * 2;      // P tile, bf16, [head][64] 128B-swizzled (PV operand A)
 constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, bf16
-// TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64; P(c) overwrites
-// the first 32 columns of S(c) as bf16 pairs) | Q (bf16 pairs, 128)
+// TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64) | Q (bf16 pairs, 128)
 constexpr uint32_t kOCol = 0, kSCol = 256, kQCol = 384;
 constexpr int kSoftWarps = 8;                  // warps 0..7
 constexpr int kSendWarp0 = 8, kSendWarps = 4;  // warps 8..11
-constexpr int kProdWarp0 = 12, kProdWarps = 7; // warps 12..18: the chunk's 16 four-row groups
-constexpr int kMmaWarpA = 19;
-constexpr int kMlaThreads = 20 * 32;           // 20 warps: 96 registers per thread
+#ifndef MLA_PROD_WARPS
+#define MLA_PROD_WARPS 6
+#endif
+constexpr int kProdWarp0 = 12, kProdWarps = MLA_PROD_WARPS;  // the chunk's 16 four-row groups
+constexpr int kMmaWarpA = kProdWarp0 + kProdWarps;           // lane 0 issues QK
+constexpr int kMmaWarpB = kMmaWarpA + 1;                     // lane 0 issues PV
+constexpr int kMlaThreads = (kMmaWarpB + 1) * 32;            // 20 warps: 96 registers per thread
 constexpr float kRescaleThresh = 8.0f;          // log2 units
 constexpr int kPairBarBase = 2;                 // named barriers 2..5 and 6..9: the two softmax warps of a quadrant
 constexpr int kSendBar = 10;                    // named barrier 10: the sender warps
 
 struct MlaBars {
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], s_free[2];  // S tile computed / read by the softmax and sender warps
+  uint64_t p_full, pv_done;       // P tile written / PV finished reading it (one phase per chunk)
   uint64_t o_full, o_free, q_full;
   uint64_t q0_full;  // first item: Q loaded by the sender and softmax warps together
-  uint64_t x_full, x_free;  // the peer's partial tile landed / consumed
+  uint64_t x_full[2], x_free[2];  // per half of X_in: the peer's copy landed / the half consumed
   unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
   float lsum[1][2][kNH];                        // [half][head] final sums
@@ -186,8 +191,8 @@ struct MlaBars {
 };
 
 // shared memory: gather ring | the peer's partials X_in (fp32) | this CTA's
-// partials staged for the copy X_out | Q rope
-constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kQRopeBytes +
+// partials staged for the copies X_out | P | Q rope
+constexpr int kMlaSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kPBytes + kQRopeBytes +
                          static_cast<int>(sizeof(MlaBars)) + 64;
 
 struct MlaParams {
@@ -236,7 +241,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
   uint8_t* kv_smem = smem;
   uint8_t* xin_smem = kv_smem + kStages * kStageBytes;   // X_in[half]: the peer's partials
   uint8_t* xout_smem = xin_smem + kXBytes;               // X_out[half]: this CTA's, staged
-  uint8_t* qrope_smem = xout_smem + kXBytes;             // CTA1: Q[:, 512:576]
+  uint8_t* p_smem = xout_smem + kXBytes;                 // P of the current chunk
+  uint8_t* qrope_smem = p_smem + kPBytes;                // CTA1: Q[:, 512:576]
   MlaBars* bb = reinterpret_cast<MlaBars*>(qrope_smem + kQRopeBytes);
   volatile int* abort_flag = &bb->abort_flag;
 
@@ -259,15 +265,16 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bb->s_full[b], 1);
-      mbar_init(&bb->s_read[b], kSendWarps);
-      mbar_init(&bb->p_full[b], kSoftWarps);
-      mbar_init(&bb->pv_done[b], 1);
+      mbar_init(&bb->s_free[b], kSoftWarps + kSendWarps);
+      // X_in half b: the peer's bulk copy completes the phase; the phase of
+      // chunk 0 is armed here, the next one by the softmax warps of that half
+      // as they consume a chunk
+      mbar_init(&bb->x_full[b], 1);
+      mbar_init(&bb->x_free[b], kSoftWarps / 2);
+      mbar_arrive_expect_tx(&bb->x_full[b], kXHalf);
     }
-    // X_in: the peer's bulk copy completes the phase; the phase of chunk 0 is
-    // armed here, the next one by the softmax as it consumes a chunk
-    mbar_init(&bb->x_full, 1);
-    mbar_init(&bb->x_free, kSoftWarps);
-    mbar_arrive_expect_tx(&bb->x_full, kXBytes);
+    mbar_init(&bb->p_full, kSoftWarps);
+    mbar_init(&bb->pv_done, 1);
     mbar_init(&bb->o_full, 1);
     mbar_init(&bb->o_free, kSoftWarps);
     mbar_init(&bb->q_full, kSendWarps);
@@ -292,11 +299,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     // ------------------------------------------------------------ gather
     // TMA gather4 of the chunk's selected latent rows into the 128B-swizzled
     // slab layout the UMMAs read.  Gather throughput grows with the number of
-    // issuing warps, so 7 warps share each chunk's 16 four-row groups: warp pw
-    // owns groups pw, pw + 7 and pw + 14 (when < 16); lane i issues group
-    // pw + 7i over all slabs after lanes 4i..4i+3 fetched its row indices.
+    // issuing warps, so kProdWarps warps share each chunk's 16 four-row groups:
+    // warp pw owns groups pw + kProdWarps * i (i = 0, 1, 2, when < 16); lane i
+    // issues group pw + kProdWarps * i over all slabs after lanes 4i..4i+3
+    // fetched its row indices.
     const int pw = warp - kProdWarp0;
-    const int n_groups = pw + 14 < 16 ? 3 : 2;
+    const int n_groups = pw + 2 * kProdWarps < 16 ? 3 : 2;
     uint32_t g = 0;  // global chunk counter
     bool ok = true;
     for (int item = pair; item < n_items && ok; item += n_pairs) {
@@ -304,7 +312,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       if (it.n == 0) continue;
       const int32_t* irow = p.idx + static_cast<size_t>(it.row) * p.k;
       const int row_base = it.kv_row0;
-      const int my_group = pw + 7 * (lane >> 2);            // group whose row this lane fetches
+      const int my_group = pw + kProdWarps * (lane >> 2);   // group whose row this lane fetches
       auto fetch = [&](int c) -> int {
         const int r = c * kChunk + my_group * 4 + (lane & 3);
         return ((lane >> 2) < n_groups && r < it.nv) ? __ldg(irow + r) : -1;
@@ -333,7 +341,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
         const bool w = __all_sync(0xffffffffu, mbar_wait(&bb->kv_empty[stage], ph ^ 1, abort_flag));
         if (!w) { ok = false; break; }  // warp-uniform
         if (lane < n_groups) {
-          const int grp = pw + 7 * lane;
+          const int grp = pw + kProdWarps * lane;
           bb->kvmask[stage][grp] = static_cast<unsigned char>((m >> (4 * lane)) & 0xFu);
           uint8_t* dst = kv_smem + stage * kStageBytes + grp * 512;
           mbar_arrive_expect_tx(&bb->kv_full[stage], n_slabs * 512);
@@ -343,31 +351,14 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       }
     }
   } else if (warp == kMmaWarpA) {
-    // ------------------------------------------------------------ MMA
+    // ------------------------------------------------------------ MMA: QK
+    // S[g & 1] = Q K(g)^T as soon as the chunk's rows have landed and the
+    // softmax and sender warps have read S(g - 2) out of that buffer.
     if (lane == 0) {
       uint32_t g = 0, it_n = 0;
       bool ok = true;
       const uint32_t idesc_qk = make_idesc_bf16(128, kChunk, 0, 0);
-      const uint32_t idesc_pv = make_idesc_bf16(128, 256, 0, 1);
       const uint32_t qrope_base = smem_u32(qrope_smem);
-      auto issue_pv = [&](uint32_t gc, bool first) -> bool {
-        const int sb = gc & 1;
-        if (!mbar_wait(&bb->p_full[sb], (gc >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const int stage = gc % kStages;
-        // V = this CTA's slabs 0..3: value columns 0..255 (CTA0) or 256..511 (CTA1);
-        // A = P(gc) (bf16) in the first 32 TMEM columns of S[gc & 1]
-        const uint32_t v_base = smem_u32(kv_smem + stage * kStageBytes);
-        const uint32_t p_col = kSCol + sb * 64;
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-          const uint64_t bd = make_smem_desc(v_base + kk * 2048, kSlabBytes, 1024, kSwizzle128B);
-          umma_bf16_ts(tmem + kOCol, tmem + p_col + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&bb->pv_done[sb]);
-        umma_commit(&bb->kv_empty[stage]);
-        return true;
-      };
       for (int item = pair; item < n_items && ok; item += n_pairs) {
         const MlaItem it = mla_item(p, item);
         if (it.n == 0) continue;
@@ -376,11 +367,14 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           break;
         }
         tc_fence_after();
-        for (int c = 0; c < it.n && ok; ++c, ++g) {
+        for (int c = 0; c < it.n; ++c, ++g) {
           const int stage = g % kStages;
-          if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag) ||
+              !mbar_wait(&bb->s_free[g & 1], ((g >> 1) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          // S[g & 1] was last read by PV(g - 2), issued before this QK (in-order)
           const uint32_t kb = smem_u32(kv_smem + stage * kStageBytes);
           const uint32_t s_col = kSCol + (g & 1) * 64;
 #pragma unroll
@@ -399,14 +393,41 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             }
           }
           umma_commit(&bb->s_full[g & 1]);
-          if (c >= 1) {
-            if (c == 1 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag)) { ok = false; break; }
-            if (!issue_pv(g - 1, c == 1)) { ok = false; break; }
+        }
+        ++it_n;
+      }
+    }
+  } else if (warp == kMmaWarpB) {
+    // ------------------------------------------------------------ MMA: PV
+    // O += P(g) V(g), P (bf16) from shared memory, V = this CTA's slabs 0..3:
+    // value columns 0..255 (CTA0) or 256..511 (CTA1).
+    if (lane == 0) {
+      uint32_t g = 0, it_n = 0;
+      bool ok = true;
+      const uint32_t idesc_pv = make_idesc_bf16(128, 256, 0, 1);
+      const uint32_t p_base = smem_u32(p_smem);
+      for (int item = pair; item < n_items && ok; item += n_pairs) {
+        const MlaItem it = mla_item(p, item);
+        if (it.n == 0) continue;
+        for (int c = 0; c < it.n; ++c, ++g) {
+          const int stage = g % kStages;
+          if (!mbar_wait(&bb->p_full, g & 1, abort_flag) ||
+              (c == 0 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(kv_smem + stage * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            const uint64_t ad = make_smem_desc(p_base + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = make_smem_desc(v_base + kk * 2048, kSlabBytes, 1024, kSwizzle128B);
+            umma_bf16_ss(tmem + kOCol, ad, bd, idesc_pv, (c == 0 && kk == 0) ? 0u : 1u);
+          }
+          umma_commit(&bb->pv_done);
+          umma_commit(&bb->kv_empty[stage]);
         }
         if (!ok) break;
-        if (it.n == 1 && !mbar_wait(&bb->o_free, (it_n & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (!issue_pv(g - 1, it.n == 1)) { ok = false; break; }
         umma_commit(&bb->o_full);
         ++it_n;
       }
@@ -421,7 +442,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int stid = threadIdx.x - kSendWarp0 * 32;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const uint32_t xin_remote = mapa_shared(smem_u32(xin_smem), peer);
-    const uint32_t xfull_remote = mapa_shared(smem_u32(&bb->x_full), peer);
+    const uint32_t xfull_remote0 = mapa_shared(smem_u32(&bb->x_full[0]), peer);
+    const uint32_t xfull_remote1 = mapa_shared(smem_u32(&bb->x_full[1]), peer);
     // A failed (timed-out) wait only clears `ok`; the sender warps leave their
     // loops together, at the next named barrier, so none is left waiting there.
     uint32_t g = 0, it_n = 0;
@@ -437,17 +459,27 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       if (ok) {
         const uint4* qsrc = reinterpret_cast<const uint4*>(
             p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0);
+        // two 32-column blocks per round, all their loads in flight at once;
         // the first item's blocks 1 and 2 are loaded by the softmax warps
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
-          if (it_n == 0 && (blk == 1 || blk == 2)) continue;
-          uint32_t r[32];
+        for (int b2 = 0; b2 < 4; b2 += 2) {
+          const int b0 = it_n == 0 ? 3 * (b2 >> 1) : b2;  // first item: block 0, then block 3
+          const int nb = it_n == 0 ? 1 : 2;
+          uint32_t ra[32], rb[32];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const uint4 v = __ldg(qsrc + blk * 8 + j);
-            r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+            const uint4 v = __ldg(qsrc + b0 * 8 + j);
+            ra[4 * j] = v.x; ra[4 * j + 1] = v.y; ra[4 * j + 2] = v.z; ra[4 * j + 3] = v.w;
           }
-          tmem_st32x32(t_lane + kQCol + blk * 32, r);
+          if (nb == 2) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint4 v = __ldg(qsrc + (b0 + 1) * 8 + j);
+              rb[4 * j] = v.x; rb[4 * j + 1] = v.y; rb[4 * j + 2] = v.z; rb[4 * j + 3] = v.w;
+            }
+          }
+          tmem_st32x32(t_lane + kQCol + b0 * 32, ra);
+          if (nb == 2) tmem_st32x32(t_lane + kQCol + (b0 + 1) * 32, rb);
         }
         if (rank == 1 && it_n > 0) {  // the first item's rope part: softmax warps
           // columns 512..575 -> 128B-swizzled K-major row h of the rope tile
@@ -468,14 +500,14 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
                            ? reinterpret_cast<const char*>(
                                  p.q + (static_cast<size_t>((item + n_pairs) / p.S) * kNH + h) * kDQK + col0)
                            : nullptr;
-      const int c_pf = max(0, it.n - 4);
+      const int c_pf = max(0, it.n - 8);
       for (int c = 0; c < it.n; ++c, ++g) {
         const int sb = g & 1;
         if (c == c_pf && nq != nullptr)
           for (int ln = 0; ln < (rank == 0 ? 4 : 5); ++ln) prefetch_l2(nq + ln * 128);
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_full[sb], (g >> 1) & 1, abort_flag));
         tc_fence_after();
-        // X_out is free once the previous chunk's copy has read it
+        // X_out is free once the previous chunk's copies have read it
         if (stid == 0) bulk_wait_read_all();
         ok = named_bar_and(kSendBar, kSendWarps * 32, ok);
         if (ok) {
@@ -493,18 +525,24 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
                   make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           }
         }
+        // S(g) has been read: QK(g + 2) may overwrite the buffer
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&bb->s_read[sb]);
+        if (lane == 0 && ok) mbar_arrive(&bb->s_free[sb]);
         fence_proxy_async_smem();
         named_bar_sync(kSendBar + 1, kSendWarps * 32);
         if (stid == 0 && ok) {
-          // the peer's X_in is free once its softmax has consumed chunk g-1
-          if (mbar_wait_cluster(&bb->x_free, (g & 1) ^ 1, abort_flag)) {
-            bulk_copy_to_peer(xin_remote, smem_u32(xout_smem), kXBytes, xfull_remote);
-            bulk_commit_group();
-          } else {
-            ok = false;  // the abort flag is raised; the next barrier ends the loop
+          // each half of the peer's X_in is free once the peer's softmax warps
+          // of that half have consumed chunk g - 1
+#pragma unroll 1
+          for (int half = 0; half < 2 && ok; ++half) {
+            if (mbar_wait_cluster(&bb->x_free[half], (g & 1) ^ 1, abort_flag)) {
+              bulk_copy_to_peer(xin_remote + half * kXHalf, smem_u32(xout_smem) + half * kXHalf, kXHalf,
+                                half ? xfull_remote1 : xfull_remote0);
+              bulk_commit_group();
+            } else {
+              ok = false;  // the abort flag is raised; the next barrier ends the loop
+            }
           }
         }
       }
@@ -512,7 +550,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       if (!ok) break;
       ++it_n;
     }
-    if (stid == 0) bulk_wait_read_all();  // the last copy has read the staging buffer
+    if (stid == 0) bulk_wait_read_all();  // the last copies have read the staging buffer
   } else {
     // ------------------------------------------------------------ softmax
     // thread = (head h = TMEM lane, half hf of the chunk's 64 columns)
@@ -520,7 +558,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int h = qd * 32 + lane;
     const int pair_bar = kPairBarBase + qd;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const uint32_t xfree_remote = mapa_shared(smem_u32(&bb->x_free), peer);
+    const uint32_t xfree_remote = mapa_shared(smem_u32(&bb->x_free[hf]), peer);
     // A failed (timed-out) wait only clears `ok`; the two warps of a head pair
     // leave their loops together at the next pair barrier.
     uint32_t g = 0, it_n = 0;
@@ -586,8 +624,23 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
 #pragma unroll
           for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
         }
+        // S(g) has been read: QK(g + 2) may overwrite the buffer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&bb->s_free[sb]);
+        // the rows' validity bits (eight 4-bit group masks, one per byte ->
+        // 32 row bits), read while the peer's partials are in flight
+        if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
+        uint32_t vm = 0xFFFFFFFFu;
+        if (ok) {
+          uint64_t x = *reinterpret_cast<const uint64_t*>(&bb->kvmask[stage][8 * hf]) & 0x0F0F0F0F0F0F0F0Full;
+          x = (x | (x >> 4)) & 0x00FF00FF00FF00FFull;
+          x = (x | (x >> 8)) & 0x0000FFFF0000FFFFull;
+          x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
+          vm = static_cast<uint32_t>(x);
+        }
         // + the peer's partial scores of the same columns (fp32)
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_full, g & 1, abort_flag));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_full[hf], g & 1, abort_flag));
         if (ok) {
           const uint8_t* xr = xin_smem + hf * kXHalf + h * 128;
 #pragma unroll
@@ -599,21 +652,14 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
             s[4 * j + 3] += o.w;
           }
         }
-        // X_in is consumed (the additions above used every loaded value):
-        // arm the phase of the next chunk, then let the peer send it
+        // this half of X_in is consumed (the additions above used every loaded
+        // value): arm its phase for the next chunk, then let the peer send it
         __syncwarp();
-        if (threadIdx.x == 0 && ok) mbar_arrive_expect_tx(&bb->x_full, kXBytes);
+        if (qd == 0 && lane == 0 && ok) mbar_arrive_expect_tx(&bb->x_full[hf], kXHalf);
         if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote);
         // mask, scale, chunk max (combined with the other half of the head)
-        if (ok) ok = mbar_wait(&bb->kv_full[stage], (g / kStages) & 1, abort_flag);
         float lmax = -INFINITY;
         if (ok) {
-          // eight 4-bit group masks (one per byte) -> 32 row bits
-          uint64_t x = *reinterpret_cast<const uint64_t*>(&bb->kvmask[stage][8 * hf]) & 0x0F0F0F0F0F0F0F0Full;
-          x = (x | (x >> 4)) & 0x00FF00FF00FF00FFull;
-          x = (x | (x >> 8)) & 0x0000FFFF0000FFFFull;
-          x = (x | (x >> 16)) & 0x00000000FFFFFFFFull;
-          const uint32_t vm = static_cast<uint32_t>(x);
           if (vm != 0xFFFFFFFFu) {  // warp-uniform: rows are the same for every head
 #pragma unroll
             for (int j = 0; j < 32; ++j) s[j] = ((vm >> j) & 1u) ? s[j] : -INFINITY;
@@ -638,7 +684,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           const float factor = grow ? ex2_approx(m_run - cmax) : 1.f;  // 0 when m_run = -inf
           if (c > 0) {
             // O holds PV of the earlier chunks: wait for PV(g-1), scale my 128 columns
-            ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag));
+            ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
             tc_fence_after();
             if (ok) {
 #pragma unroll 1
@@ -671,17 +717,20 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         l_run += (e4[0] + e4[1]) + (e4[2] + e4[3]);
-        // P(g) overwrites the first 32 columns of S[g & 1] once the sender has
-        // read them (both halves of this head read theirs before the pair barrier)
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bb->s_read[sb], (g >> 1) & 1, abort_flag));
-        tc_fence_after();
+        // P(g) overwrites P(g - 1) once PV(g - 1) has read it: row h of the
+        // 128B-swizzled K-major tile, this half's 64 bytes as four 16-byte pieces
+        if (ok && g > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
         if (ok) {
-          tmem_st32x16(t_lane + kSCol + sb * 64 + hf * 16, pk);
-          tmem_st_wait();
+          uint8_t* prow = p_smem + h * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(prow + (((hf * 4 + i) ^ (h & 7)) << 4)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          fence_proxy_async_smem();
         }
-        tc_fence_before();
+        tc_fence_before();  // orders a rescale's TMEM stores before PV(g)
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&bb->p_full[sb]);
+        if (lane == 0 && ok) mbar_arrive(&bb->p_full);
       }
       // combine the two halves' sums
       bb->lsum[0][hf][h] = l_run;

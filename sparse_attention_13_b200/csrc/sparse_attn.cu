@@ -161,6 +161,7 @@ constexpr int kXBytes = kNH * kChunk * 4;      // partial score tile, fp32
 constexpr int kXHalf = kXBytes / 2;            // one half: 32 columns of 128 heads, [head][32] fp32
 constexpr int kPBytes = kNH * kChunk * 2;      // P tile, bf16, [head][64] 128B-swizzled (PV operand A)
 constexpr int kQRopeBytes = kNH * 128;         // CTA1: query columns 512..575, bf16
+constexpr int kQBoxBytes = kNH * 128;          // one TMA box of the query: 128 heads x 64 columns
 // TMEM columns: O (fp32, 256) | S double buffer (fp32, 2 x 64) | Q (bf16 pairs, 128)
 constexpr uint32_t kOCol = 0, kSCol = 256, kQCol = 384;
 constexpr int kSoftWarps = 8;                  // warps 0..7
@@ -181,7 +182,7 @@ struct MlaBars {
   uint64_t s_full[2], s_free[2];  // S tile computed / read by the softmax and sender warps
   uint64_t p_full, pv_done;       // P tile written / PV finished reading it (one phase per chunk)
   uint64_t o_full, o_free, q_full;
-  uint64_t q0_full;  // first item: Q loaded by the sender and softmax warps together
+  uint64_t q_tma, q_cp;  // the item's query boxes landed / copied into TMEM (two phases per item)
   uint64_t x_full[2], x_free[2];  // per half of X_in: the peer's copy landed / the half consumed
   unsigned char kvmask[kStages][16];            // per 4-row group: validity bits
   float red[2][2][kNH];                         // [parity][half][head] chunk maxima
@@ -234,7 +235,8 @@ __device__ __forceinline__ MlaItem mla_item(const MlaParams& p, int item) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
-mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParams p) {
+mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
+                       const MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -277,8 +279,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     mbar_init(&bb->pv_done, 1);
     mbar_init(&bb->o_full, 1);
     mbar_init(&bb->o_free, kSoftWarps);
-    mbar_init(&bb->q_full, kSendWarps);
-    mbar_init(&bb->q0_full, kSendWarps + kSoftWarps);
+    mbar_init(&bb->q_full, 1);
+    mbar_init(&bb->q_tma, 1);
+    mbar_init(&bb->q_cp, 1);
     bb->abort_flag = 0;
     fence_barrier_init();
   }
@@ -362,7 +365,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       for (int item = pair; item < n_items && ok; item += n_pairs) {
         const MlaItem it = mla_item(p, item);
         if (it.n == 0) continue;
-        if (!mbar_wait(it_n == 0 ? &bb->q0_full : &bb->q_full, it_n == 0 ? 0u : (it_n - 1) & 1, abort_flag)) {
+        if (!mbar_wait(&bb->q_full, it_n & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -442,6 +445,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
     const int stid = threadIdx.x - kSendWarp0 * 32;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const uint32_t xin_remote = mapa_shared(smem_u32(xin_smem), peer);
+    uint32_t q_phase = 0;  // completed phases of q_tma and q_cp
     const uint32_t xfull_remote0 = mapa_shared(smem_u32(&bb->x_full[0]), peer);
     const uint32_t xfull_remote1 = mapa_shared(smem_u32(&bb->x_full[1]), peer);
     // A failed (timed-out) wait only clears `ok`; the sender warps leave their
@@ -453,47 +457,41 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
       if (it.n == 0) continue;
       // Q's TMEM columns (and CTA1's rope tile) are free: this warp saw the
       // previous item's last S, so every QK of that item has completed (no
-      // later MMA of it reads Q).  The load overlaps that item's last
-      // softmax, PV and epilogue.
+      // later MMA of it reads Q).  One thread brings the CTA's query part in:
+      // TMA boxes of 128 heads x 64 columns (128B-swizzled, two at a time
+      // through the idle staging buffer X_out) and tcgen05.cp into TMEM, in
+      // the layout the QK MMA reads; CTA1's rope columns land directly in
+      // their shared-memory tile.  The load overlaps the item's last softmax,
+      // PV and epilogue.
       tc_fence_after();
-      if (ok) {
-        const uint4* qsrc = reinterpret_cast<const uint4*>(
-            p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0);
-        // two 32-column blocks per round, all their loads in flight at once;
-        // the first item's blocks 1 and 2 are loaded by the softmax warps
+      if (stid == 0 && ok) {
+        bulk_wait_read_all();  // the previous chunk's copies have read X_out
+        const int qrow = it.row * kNH;
 #pragma unroll 1
-        for (int b2 = 0; b2 < 4; b2 += 2) {
-          const int b0 = it_n == 0 ? 3 * (b2 >> 1) : b2;  // first item: block 0, then block 3
-          const int nb = it_n == 0 ? 1 : 2;
-          uint32_t ra[32], rb[32];
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          const uint32_t bytes = 2 * kQBoxBytes + (rank == 1 && pass == 0 ? kQRopeBytes : 0);
+          mbar_arrive_expect_tx(&bb->q_tma, bytes);
+          for (int b = 0; b < 2; ++b)
+            tma_load_2d(xout_smem + b * kQBoxBytes, &tm_q, &bb->q_tma, col0 + (2 * pass + b) * 64, qrow);
+          if (rank == 1 && pass == 0) tma_load_2d(qrope_smem, &tm_q, &bb->q_tma, 512, qrow);
+          ok = mbar_wait(&bb->q_tma, q_phase & 1, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 v = __ldg(qsrc + b0 * 8 + j);
-            ra[4 * j] = v.x; ra[4 * j + 1] = v.y; ra[4 * j + 2] = v.z; ra[4 * j + 3] = v.w;
+              for (int kk = 0; kk < 4; ++kk)
+                tc_cp_128x256b(tmem + kQCol + (2 * pass + b) * 32 + kk * 8,
+                               make_smem_desc(smem_u32(xout_smem + b * kQBoxBytes) + kk * 32, 16, 1024,
+                                              kSwizzle128B));
+            umma_commit(&bb->q_cp);
+            ok = mbar_wait(&bb->q_cp, q_phase & 1, abort_flag);  // X_out read, TMEM written
           }
-          if (nb == 2) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint4 v = __ldg(qsrc + (b0 + 1) * 8 + j);
-              rb[4 * j] = v.x; rb[4 * j + 1] = v.y; rb[4 * j + 2] = v.z; rb[4 * j + 3] = v.w;
-            }
-          }
-          tmem_st32x32(t_lane + kQCol + b0 * 32, ra);
-          if (nb == 2) tmem_st32x32(t_lane + kQCol + (b0 + 1) * 32, rb);
+          ++q_phase;
         }
-        if (rank == 1 && it_n > 0) {  // the first item's rope part: softmax warps
-          // columns 512..575 -> 128B-swizzled K-major row h of the rope tile
-          uint8_t* dst = qrope_smem + h * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(dst + ((j ^ (h & 7)) << 4)) = __ldg(qsrc + 32 + j);
-          fence_proxy_async_smem();
-        }
-        tmem_st_wait();
+        tc_fence_before();
+        if (ok) mbar_arrive(&bb->q_full);
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(it_n == 0 ? &bb->q0_full : &bb->q_full);
       // this head's part of the next item's query, warmed into L2 a few chunks
       // before it is loaded (earlier, the gathers would evict it again)
       const char* nq = item + n_pairs < n_items
@@ -578,35 +576,6 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const MlaParam
           if (p.lse && rank == 0 && hf == 0) p.lse[static_cast<size_t>(it.row) * kNH + h] = -INFINITY;
         }
         continue;
-      }
-      if (it_n == 0) {
-        // first item: query block 1 + hf of this head (and, in CTA1, its rope
-        // columns), loaded alongside the sender's blocks 0 and 3 so that the
-        // first QK starts sooner
-        if (ok) {
-          const uint4* qsrc = reinterpret_cast<const uint4*>(
-              p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0) + (1 + hf) * 8;
-          uint32_t ra[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 a = __ldg(qsrc + j);
-            ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
-          }
-          tmem_st32x32(t_lane + kQCol + (1 + hf) * 32, ra);
-          if (rank == 1 && hf == 0) {
-            // CTA1: query columns 512..575 -> 128B-swizzled row h of the rope tile
-            uint8_t* dst = qrope_smem + h * 128;
-            const uint4* rsrc = reinterpret_cast<const uint4*>(
-                p.q + (static_cast<size_t>(it.row) * kNH + h) * kDQK + col0) + 32;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + ((j ^ (h & 7)) << 4)) = __ldg(rsrc + j);
-            fence_proxy_async_smem();
-          }
-          tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&bb->q0_full);
       }
       // l_run: softmax denominator (fp32, before the bf16 rounding of P); each
       // half of a head keeps the sum of its own columns.
@@ -918,10 +887,14 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     if (rows * sp.S > (1ll << 31) - 1) return set_error(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn: too many rows");
     const size_t need = sp.S > 1 ? static_cast<size_t>(rows) * sp.S * kNH * (kDV / 2 + 1) * 4 : 0;
     if (need > ws_bytes || (need && !ws)) return set_error(DSA_ERR_WORKSPACE, "dsa_sparse_attn: workspace too small");
-    CUtensorMap tkv;
+    CUtensorMap tkv, tq;
     if (!encode_tiled_2d(&tkv, kbuf, kDQK, static_cast<uint64_t>(kv_rows),
                          static_cast<uint64_t>(k_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
       return set_error(DSA_ERR_CUDA, "tensor map for the latent cache failed");
+    // the query as [rows * 128 heads][576] with boxes of 128 heads x 64 columns
+    if (!encode_tiled_2d(&tq, q, kDQK, static_cast<uint64_t>(rows) * kNH, kDQK * 2, 64, kNH,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+      return set_error(DSA_ERR_CUDA, "tensor map for the query failed");
     MlaParams p{};
     p.q = reinterpret_cast<const __nv_bfloat16*>(q);
     p.idx = idx;
@@ -943,7 +916,7 @@ dsa_status sparse_attn_launch(const dsa_bf16* q, const dsa_bf16* kbuf, int64_t k
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(mla_sparse_attn_kernel), kMlaSmem);
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla smem attribute: ") + cudaGetErrorString(e));
     e = launch_pdl(mla_sparse_attn_kernel, dim3(static_cast<unsigned>(2 * sp.pairs)), dim3(kMlaThreads), kMlaSmem,
-                   stream, tkv, p);
+                   stream, tkv, tq, p);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(DSA_ERR_CUDA, std::string("mla launch: ") + cudaGetErrorString(e));
     if (sp.S > 1) {

@@ -626,6 +626,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
         __syncwarp();
         if (qd == 0 && lane == 0 && ok) mbar_arrive_expect_tx(&bb->x_full[hf], kXHalf);
         if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote);
+        // PV(g - 1) has read P(g - 1) (and O holds it): checked here, off the
+        // chain of waits that follows, before P(g) and any rescale of O
+        if (ok && g > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
         // mask, scale, chunk max (combined with the other half of the head)
         float lmax = -INFINITY;
         if (ok) {
@@ -652,8 +655,8 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
         if (__any_sync(0xffffffffu, grow)) {
           const float factor = grow ? ex2_approx(m_run - cmax) : 1.f;  // 0 when m_run = -inf
           if (c > 0) {
-            // O holds PV of the earlier chunks: wait for PV(g-1), scale my 128 columns
-            ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
+            // O holds PV of the earlier chunks (PV(g - 1) has completed: see
+            // above): scale my 128 columns
             tc_fence_after();
             if (ok) {
 #pragma unroll 1
@@ -686,9 +689,9 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
           pk[j] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         l_run += (e4[0] + e4[1]) + (e4[2] + e4[3]);
-        // P(g) overwrites P(g - 1) once PV(g - 1) has read it: row h of the
-        // 128B-swizzled K-major tile, this half's 64 bytes as four 16-byte pieces
-        if (ok && g > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
+        // P(g) overwrites P(g - 1), which PV(g - 1) has read (checked above):
+        // row h of the 128B-swizzled K-major tile, this half's 64 bytes as
+        // four 16-byte pieces
         if (ok) {
           uint8_t* prow = p_smem + h * 128;
 #pragma unroll

@@ -609,6 +609,7 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
           vm = static_cast<uint32_t>(x);
         }
         // + the peer's partial scores of the same columns (fp32)
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bb->x_full[hf], g & 1, abort_flag));
         if (ok) {
           const uint8_t* xr = xin_smem + hf * kXHalf + h * 128;
@@ -619,6 +620,12 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
             s[4 * j + 1] += o.y;
             s[4 * j + 2] += o.z;
             s[4 * j + 3] += o.w;
+            // the raw maximum of a fully valid chunk, in four chains while
+            // the loads are in flight
+            m4[0] = fmaxf(m4[0], s[4 * j]);
+            m4[1] = fmaxf(m4[1], s[4 * j + 1]);
+            m4[2] = fmaxf(m4[2], s[4 * j + 2]);
+            m4[3] = fmaxf(m4[3], s[4 * j + 3]);
           }
         }
         // this half of X_in is consumed (the additions above used every loaded
@@ -626,25 +633,28 @@ mla_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_c
         __syncwarp();
         if (qd == 0 && lane == 0 && ok) mbar_arrive_expect_tx(&bb->x_full[hf], kXHalf);
         if (lane == 0 && ok) mbar_arrive_remote_relaxed(xfree_remote);
-        // PV(g - 1) has read P(g - 1) (and O holds it): checked here, off the
-        // chain of waits that follows, before P(g) and any rescale of O
-        if (ok && g > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
-        // mask, scale, chunk max (combined with the other half of the head)
+        // mask, scale, chunk max (combined with the other half of the head);
+        // the scale (> 0) is applied to the maximum and inside the exponent
+        // with one FMA per element
         float lmax = -INFINITY;
         if (ok) {
           if (vm != 0xFFFFFFFFu) {  // warp-uniform: rows are the same for every head
 #pragma unroll
             for (int j = 0; j < 32; ++j) s[j] = ((vm >> j) & 1u) ? s[j] : -INFINITY;
-          }
-          // max of the raw scores as a tree (short dependency chains); the
-          // scale (> 0) is applied to the maximum and inside the exponent
-          // with one FMA per element
-          float m8[8];
+            // max of the masked scores as a tree (short dependency chains)
+            float m8[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) m8[j] = fmaxf(fmaxf(s[j], s[j + 8]), fmaxf(s[j + 16], s[j + 24]));
-          lmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            for (int j = 0; j < 8; ++j) m8[j] = fmaxf(fmaxf(s[j], s[j + 8]), fmaxf(s[j + 16], s[j + 24]));
+            lmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          } else {
+            lmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          }
         }
         bb->red[g & 1][hf][h] = lmax;
+        // PV(g - 1) has read P(g - 1) (and O holds it): checked while the
+        // other half of the head reaches the pair barrier, before P(g) and
+        // any rescale of O
+        if (ok && g > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bb->pv_done, (g - 1) & 1, abort_flag));
         ok = named_bar_and(pair_bar, 64, ok);
         if (!ok) break;
         const float cmax = fmaxf(lmax, bb->red[g & 1][hf ^ 1][h]) * p.scale_log2;

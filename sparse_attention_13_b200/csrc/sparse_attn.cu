@@ -800,6 +800,21 @@ mla_merge_kernel(const uint32_t* __restrict__ part_o, const float* __restrict__ 
   __shared__ float wgt[kMaxMergeSplits][kNH];
   __shared__ uint32_t tile[kNH][kMergeCols / 2 + 1];
   const int t = threadIdx.x;
+  constexpr int kPairs = kMergeCols / 4;  // column pairs per thread (two threads per head)
+  const int h = t & (kNH - 1), half = t >> 7;
+  const int cp0 = cb * (kMergeCols / 2) + half * kPairs;
+  // the first kPre splits' partial words are loaded before the weights are
+  // known, so that both global round trips overlap
+  constexpr int kPre = 8;
+  uint32_t pre[kPre][kPairs];
+#pragma unroll
+  for (int j = 0; j < kPre; ++j) {
+    if (j < S) {
+      const uint32_t* src = part_o + ((row * S + j) * 256 + cp0) * kNH + h;
+#pragma unroll
+      for (int i = 0; i < kPairs; ++i) pre[j][i] = src[i * kNH];
+    }
+  }
   for (int e = t; e < S * kNH; e += kMergeThreads) wgt[e / kNH][e % kNH] = part_lse[row * S * kNH + e];
   __syncthreads();
   if (t < kNH) {
@@ -816,14 +831,23 @@ mla_merge_kernel(const uint32_t* __restrict__ part_o, const float* __restrict__ 
     if (lse && cb == 0) lse[row * kNH + t] = z > 0.f ? m + __logf(z) : -INFINITY;
   }
   __syncthreads();
-  constexpr int kPairs = kMergeCols / 4;  // column pairs per thread (two threads per head)
-  const int h = t & (kNH - 1), half = t >> 7;
-  const int cp0 = cb * (kMergeCols / 2) + half * kPairs;
   float acc[2 * kPairs];
 #pragma unroll
   for (int i = 0; i < 2 * kPairs; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kPre; ++j) {
+    if (j < S) {
+      const float wj = wgt[j][h];
+#pragma unroll
+      for (int i = 0; i < kPairs; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pre[j][i]));
+        acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+      }
+    }
+  }
 #pragma unroll 4
-  for (int j = 0; j < S; ++j) {
+  for (int j = kPre; j < S; ++j) {
     const float wj = wgt[j][h];
     const uint32_t* src = part_o + ((row * S + j) * 256 + cp0) * kNH + h;
     uint32_t wv[kPairs];

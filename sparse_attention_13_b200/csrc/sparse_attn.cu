@@ -9,30 +9,32 @@
 //   A cluster of two CTAs owns one query row (or one key-range split of it)
 //   at a time.  CTA0 holds latent columns 0..255 of the query in TMEM, CTA1
 //   columns 256..511 in TMEM and 512..575 in shared memory (the A operands of
-//   the QK UMMAs); CTA c accumulates output
-//   columns 256c..256c+255 in TMEM (fp32).  Per chunk of 64 selected rows:
-//     7 producer warps  TMA gather4 of the chunk's latent rows (CTA0: 4 slabs
+//   the QK UMMAs); CTA c accumulates output columns 256c..256c+255 in TMEM
+//   (fp32).  Per chunk of 64 selected rows:
+//     6 producer warps  TMA gather4 of the chunk's latent rows (CTA0: 4 slabs
 //                    of 64 columns, CTA1: 5 slabs) into the 128B-swizzled
 //                    layout, 3-stage ring; each selected row is read from
 //                    memory exactly once;
-//     MMA warp       S_c = Q_c K_c^T over the CTA's columns (A from TMEM) into
-//                    a double-buffered S tile, then, one chunk behind,
-//                    O_c += P V_c with P read from TMEM and V_c the gathered
-//                    slabs 0..3 read as an MN-major B operand;
+//     QK thread      S_c = Q_c K_c^T over the CTA's columns (A from TMEM) into
+//                    a double-buffered S tile, as soon as the rows have
+//                    landed and S two chunks back has been read;
+//     PV thread      O_c += P V_c, P (bf16) from shared memory, V_c the
+//                    gathered slabs 0..3 read as an MN-major B operand;
 //     4 sender warps (thread = head) read S_c as soon as QK completes,
-//                    stage it, fp32, in shared memory and ship it to the peer
-//                    with one bulk copy into the peer's shared memory
-//                    (tx-counted on its mbarrier; the peer frees the tile as
-//                    soon as its softmax has read it); they also load the
-//                    next row's query into TMEM as soon as the last QK of the
-//                    current row has completed;
+//                    stage it, fp32, in shared memory and ship each 16 KB
+//                    half to the peer with one bulk copy as soon as it is
+//                    staged (tx-counted on the peer's mbarrier of that half;
+//                    the peer frees a half as soon as its softmax has read
+//                    it); one of them loads the next row's query (TMA boxes
+//                    through the staging tile, tcgen05.cp into TMEM) as soon
+//                    as the last QK of the current row has completed;
 //     8 softmax warps (thread = head = TMEM lane x half of the chunk) add the
 //                    peer's partial (S = S_0 + S_1, identical in both CTAs as
 //                    fp32 addition commutes), mask padded rows (fully valid
 //                    chunks skip it), run the online softmax in the log2
 //                    domain with lazy rescaling of O (only when the running
-//                    max grows by more than 2^8), and write P as bf16 over the
-//                    first 32 columns of S_c in TMEM.
+//                    max grows by more than 2^8), and write P as bf16 into a
+//                    128B-swizzled K-major tile in shared memory.
 //   The finished row is normalised by the softmax sum and stored as bf16.
 //   Few long rows (decode) split the index list across clusters; the
 //   partials (normalised O as bf16 pairs in a head-minor layout, so that the

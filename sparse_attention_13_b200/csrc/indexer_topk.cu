@@ -99,6 +99,7 @@ struct SelShared {
   int wcnt[kSelRows][kEpiWarps];
   int woff[kSelRows][kEpiWarps];
   int sel_bin, kk_new, bin_count, total;
+  uint32_t wlo[kEpiWarps], whi[kEpiWarps];  // per-warp key range
   unsigned long long minval;
 };
 
@@ -255,10 +256,39 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
   uint32_t thr = 0u;       // threshold score key
   int ties = 1 << 30;      // how many entries equal to thr are kept (in order)
   if (cnt > k) {
-    uint32_t prefix = 0u;
+    // The bits above the highest one in which the smallest and the largest key
+    // differ are common to all entries, so the radix starts at that bit: the
+    // first digit spreads the entries over the bins instead of piling them into
+    // the one or two bins of a shared exponent, and the passes over common
+    // bits are skipped.
+    uint32_t lo = ~0u, hi = 0u;
+#pragma unroll
+    for (int r = 0; r < kSelRows; ++r) {
+      const uint32_t key = static_cast<uint32_t>(v[r] >> 32);
+      if (r * kEpiThreads + tid < cnt) {
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+      }
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) { sh.wlo[warp] = lo; sh.whi[warp] = hi; }
+    named_bar_sync(kEpiBar, kEpiThreads);
+#pragma unroll
+    for (int w = 0; w < kEpiWarps; ++w) {
+      lo = sh.wlo[w] < lo ? sh.wlo[w] : lo;
+      hi = sh.whi[w] > hi ? sh.whi[w] : hi;
+    }
+    const uint32_t diff = lo ^ hi;
+    const int hb = diff ? 31 - __clz(diff) : -1;   // highest differing bit
+    uint32_t prefix = hb < 0 ? hi : hi & ~((2u << hb) - 1u);  // hb = 31: 2u << 31 wraps to 0
     int kk = k;
     bool exact = true;     // the loop ran down to a single key value
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = hb - 7; hb >= 0;) {
+      int width = 8;
+      if (shift < 0) { width += shift; shift = 0; }
+      const int top = shift + width;               // bits >= top are fixed by prefix
+      const uint32_t dmask = (1u << width) - 1u;
       if (tid < 256) sh.hist[tid] = 0;
       named_bar_sync(kEpiBar, kEpiThreads);
 #pragma unroll
@@ -266,8 +296,8 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
         const int e = r * kEpiThreads + tid;
         if (e < cnt) {
           const uint32_t key = static_cast<uint32_t>(v[r] >> 32);
-          if (shift == 24 || (key >> (shift + 8)) == (prefix >> (shift + 8)))
-            atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+          if (top == 32 || (key >> top) == (prefix >> top))
+            atomicAdd(&sh.hist[(key >> shift) & dmask], 1);
         }
       }
       named_bar_sync(kEpiBar, kEpiThreads);
@@ -300,8 +330,10 @@ __device__ unsigned long long select_topk(const uint64_t* src, uint64_t* dst_inp
         exact = false;
         break;
       }
+      if (shift == 0) break;
+      shift -= 8;
     }
-    thr = prefix;
+    thr = prefix;          // hb < 0: every key equals hi, the first k are kept
     if (exact) ties = kk;
   }
   // keep decision: key > thr, or key == thr within the first `ties` such entries
